@@ -1,0 +1,132 @@
+"""Seeded synthetic inputs for one GQA decode step.
+
+This module draws random numbers and lays them out; it does none of the attention arithmetic.
+The CUDA path and the CPU oracle are both fed from it, so both see identical bytes.
+
+Recipe (all draws from one ``torch.Generator('cpu')`` seeded with the workload's seed):
+  1. q        [B, H_q, d]            ~ N(0, 1) * q_std
+  2. k_cache  [B, L_max, H_kv, d]    ~ N(0, 1) * kv_std, drawn one sequence (b) at a time
+  3. v_cache  [B, L_max, H_kv, d]    same
+  4. k_new    [B, H_kv, d]           ~ N(0, 1) * kv_std
+  5. v_new    [B, H_kv, d]           same
+  6. lengths  [B]  either the fixed length, or uniform integers in [1, L_max] (ragged)
+Each float is drawn in fp32 and rounded to the storage dtype with round-to-nearest-even.
+``lengths`` is the number of rows attended AFTER this step's append, so the cache starts with
+``seq_lens = lengths - 1`` and the append writes row ``lengths - 1``.  Cache rows at or beyond
+``lengths - 1`` hold no data the step may read; ``poison=True`` fills them with NaN so a kernel
+that reads them poisons its output.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    H_q: int
+    H_kv: int
+    d: int
+    L_max: int
+    dtype: torch.dtype
+    q_std: float
+    kv_std: float
+    seed: int
+    length: int | None = None          # fixed attended length; None = ragged U{1..L_max}
+    scale: float | None = None         # None = 1/sqrt(d)
+    note: str = field(default="", compare=False)
+
+    @property
+    def softmax_scale(self) -> float:
+        return self.scale if self.scale is not None else 1.0 / math.sqrt(self.d)
+
+    @property
+    def elem_bytes(self) -> int:
+        return torch.tensor([], dtype=self.dtype).element_size()
+
+
+# The pages' workloads, each named by what it is.
+WORKLOADS = {
+    w.name: w for w in [
+        Workload("tiny_fp32", B=1, H_q=8, H_kv=2, d=64, L_max=256, dtype=torch.float32,
+                 q_std=1.0, kv_std=1.0, seed=0, length=256, scale=1.0 / 8.0,
+                 note="tiny GQA step, group size 4"),
+        Workload("llama2_70b_layer", B=16, H_q=64, H_kv=8, d=128, L_max=4096,
+                 dtype=torch.bfloat16, q_std=0.5, kv_std=0.5, seed=1, length=4096,
+                 note="Llama-2-70B-shaped attention layer, GQA-8"),
+        Workload("t5xxl_g64_mha", B=32, H_q=64, H_kv=64, d=64, L_max=2048,
+                 dtype=torch.bfloat16, q_std=1.0, kv_std=1.0, seed=2, length=2048,
+                 scale=1.0 / 8.0, note="T5-XXL-shaped head sweep, G=64 (MHA)"),
+        Workload("t5xxl_g8", B=32, H_q=64, H_kv=8, d=64, L_max=2048,
+                 dtype=torch.bfloat16, q_std=1.0, kv_std=1.0, seed=2, length=2048,
+                 scale=1.0 / 8.0, note="T5-XXL-shaped head sweep, G=8"),
+        Workload("t5xxl_g1_mqa", B=32, H_q=64, H_kv=1, d=64, L_max=2048,
+                 dtype=torch.bfloat16, q_std=1.0, kv_std=1.0, seed=2, length=2048,
+                 scale=1.0 / 8.0, note="T5-XXL-shaped head sweep, G=1 (MQA)"),
+        Workload("mqa_long", B=64, H_q=32, H_kv=1, d=128, L_max=8192, dtype=torch.bfloat16,
+                 q_std=0.5, kv_std=1.0, seed=3, length=8192,
+                 note="MQA with a long cache"),
+        Workload("ragged_long", B=32, H_q=32, H_kv=8, d=128, L_max=32768, dtype=torch.bfloat16,
+                 q_std=1.0, kv_std=1.0, seed=4, length=None,
+                 note="ragged long-context batch, lengths uniform in [1, 32768]"),
+    ]
+}
+
+
+def custom(name="custom", *, B, H_q, H_kv, d, L_max, dtype=torch.bfloat16, q_std=1.0,
+           kv_std=1.0, seed=1234, length=None, scale=None) -> Workload:
+    return Workload(name, B=B, H_q=H_q, H_kv=H_kv, d=d, L_max=L_max, dtype=dtype, q_std=q_std,
+                    kv_std=kv_std, seed=seed, length=length, scale=scale)
+
+
+def _normal(shape, gen, std, dtype):
+    x = torch.randn(shape, generator=gen, dtype=torch.float32)
+    if std != 1.0:
+        x.mul_(std)
+    return x.to(dtype)
+
+
+def make_inputs(w: Workload, lengths=None, poison: bool = False) -> dict:
+    """Host (CPU) tensors for one append + decode step of workload ``w``.
+
+    ``lengths`` (a list of B ints in [0, L_max]) overrides the drawn lengths; a length of 0
+    means "no append, nothing to attend" for tests of the empty case (seq_lens starts at 0 and
+    the caller skips the append).
+    """
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed)
+    q = _normal((w.B, w.H_q, w.d), g, w.q_std, w.dtype)
+    k_cache = torch.empty((w.B, w.L_max, w.H_kv, w.d), dtype=w.dtype)
+    v_cache = torch.empty_like(k_cache)
+    for b in range(w.B):
+        k_cache[b] = _normal((w.L_max, w.H_kv, w.d), g, w.kv_std, w.dtype)
+    for b in range(w.B):
+        v_cache[b] = _normal((w.L_max, w.H_kv, w.d), g, w.kv_std, w.dtype)
+    k_new = _normal((w.B, w.H_kv, w.d), g, w.kv_std, w.dtype)
+    v_new = _normal((w.B, w.H_kv, w.d), g, w.kv_std, w.dtype)
+    if w.length is not None:
+        drawn = torch.full((w.B,), w.length, dtype=torch.int32)
+    else:
+        drawn = torch.randint(1, w.L_max + 1, (w.B,), generator=g, dtype=torch.int64).to(torch.int32)
+    if lengths is not None:
+        drawn = torch.tensor(list(lengths), dtype=torch.int32)
+        assert drawn.shape == (w.B,)
+    seq_lens_pre = torch.clamp(drawn - 1, min=0).to(torch.int32)
+    if poison:
+        nan = float("nan")
+        for b in range(w.B):
+            k_cache[b, int(seq_lens_pre[b]):] = nan
+            v_cache[b, int(seq_lens_pre[b]):] = nan
+    return {
+        "q": q, "k_cache": k_cache, "v_cache": v_cache, "k_new": k_new, "v_new": v_new,
+        "seq_lens_pre": seq_lens_pre, "lengths": drawn, "scale": w.softmax_scale,
+    }
+
+
+def ideal_kv_bytes(w: Workload, lengths) -> int:
+    """K and V bytes one decode step must read: 2 * sum(n_b) * H_kv * d * element size."""
+    return 2 * int(sum(int(n) for n in lengths)) * w.H_kv * w.d * w.elem_bytes

@@ -1,0 +1,135 @@
+"""CPU float64 oracle for one grouped-query-attention decode step.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the benchmark's CPU
+baseline leg are the only callers.  The CUDA library never imports, links or runs anything
+here, and nothing here imports the CUDA library.
+
+The arithmetic lives in ``gqa_oracle.c`` (plain C, float64); this module compiles it with gcc
+and marshals numpy arrays to it.  ``counts.py`` holds the cache-size and multiply-count
+formulas of the pages.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gqa_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+APPEND_OVERFLOW = 1
+SEQLEN_RANGE = 2
+
+
+def build(src: str = _SRC, out: str = _LIB) -> str:
+    """Compile the oracle with gcc (OpenMP over query heads, no fast-math)."""
+    cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-shared", "-fPIC", src, "-o", out, "-lm"]
+    subprocess.run(cmd, check=True)
+    return out
+
+
+def _needs_build(src: str, lib: str) -> bool:
+    return not os.path.exists(lib) or os.path.getmtime(lib) < os.path.getmtime(src)
+
+
+class Oracle:
+    """ctypes view of one compiled oracle library (the default one, or a test's variant)."""
+
+    def __init__(self, lib_path: str | None = None):
+        if lib_path is None:
+            if _needs_build(_SRC, _LIB):
+                build()
+            lib_path = _LIB
+        self.lib = ctypes.CDLL(lib_path)
+        dp = ctypes.POINTER(ctypes.c_double)
+        ip = ctypes.POINTER(ctypes.c_int32)
+        c_int = ctypes.c_int
+        self.lib.oracle_kv_append.argtypes = [dp, dp, dp, dp, ip, c_int, c_int, c_int, c_int, ip]
+        self.lib.oracle_kv_append.restype = None
+        self.lib.oracle_expand_kv.argtypes = [dp, c_int, c_int, c_int, c_int, dp]
+        self.lib.oracle_expand_kv.restype = None
+        self.lib.oracle_attend_one_head.argtypes = [dp, dp, dp, c_int, c_int, ctypes.c_size_t,
+                                                    ctypes.c_double, dp, dp]
+        self.lib.oracle_attend_one_head.restype = None
+        self.lib.oracle_gqa_decode.argtypes = [dp, dp, dp, ip, c_int, c_int, c_int, c_int, c_int,
+                                               ctypes.c_double, dp, c_int, ip]
+        self.lib.oracle_gqa_decode.restype = c_int
+        self.lib.oracle_max_threads.argtypes = []
+        self.lib.oracle_max_threads.restype = c_int
+
+    @staticmethod
+    def _f64(a) -> np.ndarray:
+        return np.ascontiguousarray(a, dtype=np.float64)
+
+    @staticmethod
+    def _dp(a: np.ndarray):
+        return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+    @staticmethod
+    def _ip(a: np.ndarray):
+        return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+
+    def max_threads(self) -> int:
+        return int(self.lib.oracle_max_threads())
+
+    def kv_append(self, k_new, v_new, k_cache, v_cache, seq_lens):
+        """Append one K/V row per (sequence, kv-head).  k_cache/v_cache ([B, L_max, H_kv, d]
+        float64) and seq_lens ([B] int32) are updated in place.  Returns the status bits."""
+        assert k_cache.dtype == np.float64 and k_cache.flags.c_contiguous
+        assert v_cache.dtype == np.float64 and v_cache.flags.c_contiguous
+        assert seq_lens.dtype == np.int32 and seq_lens.flags.c_contiguous
+        B, L_max, H_kv, d = k_cache.shape
+        kn, vn = self._f64(k_new), self._f64(v_new)
+        status = np.zeros(1, dtype=np.int32)
+        self.lib.oracle_kv_append(self._dp(kn), self._dp(vn), self._dp(k_cache), self._dp(v_cache),
+                                  self._ip(seq_lens), B, H_kv, d, L_max, self._ip(status))
+        return int(status[0])
+
+    def expand_kv(self, cache_b, n: int, H_q: int):
+        """Repeat the key/value heads of one sequence ([L_max, H_kv, d]) to [n, H_q, d]."""
+        c = self._f64(cache_b)
+        _, H_kv, d = c.shape
+        out = np.empty((n, H_q, d), dtype=np.float64)
+        self.lib.oracle_expand_kv(self._dp(c), n, H_q, H_kv, d, self._dp(out))
+        return out
+
+    def attend_one_head(self, q, K, V, scale: float):
+        """Single-head softmax attention of q [d] over rows K, V [n, d].  Returns (out, weights)."""
+        q, K, V = self._f64(q), self._f64(K), self._f64(V)
+        n, d = K.shape
+        out = np.empty(d, dtype=np.float64)
+        w = np.empty(max(n, 1), dtype=np.float64)
+        self.lib.oracle_attend_one_head(self._dp(q), self._dp(K), self._dp(V), n, d, d, scale,
+                                        self._dp(out), self._dp(w))
+        return out, w[:n]
+
+    def decode(self, q, k_cache, v_cache, seq_lens, scale: float, nthreads: int = 0,
+               return_status: bool = False):
+        """out[b, h, :] = softmax(scale * q[b,h] . K[b, :n_b, h // r]^T) . V[b, :n_b, h // r]."""
+        q, kc, vc = self._f64(q), self._f64(k_cache), self._f64(v_cache)
+        lens = np.ascontiguousarray(seq_lens, dtype=np.int32)
+        B, H_q, d = q.shape
+        Bk, L_max, H_kv, dk = kc.shape
+        assert Bk == B and dk == d and vc.shape == kc.shape and lens.shape == (B,)
+        out = np.zeros((B, H_q, d), dtype=np.float64)
+        status = np.zeros(1, dtype=np.int32)
+        rc = self.lib.oracle_gqa_decode(self._dp(q), self._dp(kc), self._dp(vc), self._ip(lens),
+                                        B, H_q, H_kv, d, L_max, float(scale), self._dp(out),
+                                        int(nthreads), self._ip(status))
+        if rc != 0:
+            raise ValueError("oracle_gqa_decode rejected the shapes (H_q % H_kv != 0?)")
+        return (out, int(status[0])) if return_status else out
+
+
+_default: Oracle | None = None
+
+
+def get() -> Oracle:
+    """The oracle compiled from ``gqa_oracle.c`` (built on first use)."""
+    global _default
+    if _default is None:
+        _default = Oracle()
+    return _default

@@ -1,0 +1,162 @@
+/*
+ * CPU oracle for one grouped-query-attention (GQA) decode step.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path loads this file: only the tests, the
+ * smoke check and the benchmark's CPU-baseline leg may call it.  It shares no code, header,
+ * table or helper with the CUDA library; inputs reach it as float64 host arrays.
+ *
+ * What it computes, and where that is stated:
+ *
+ *   - "GQA 阅读笔记" (zhongzhuzhou.org), section "GQA 架构", Algorithm 2 (GQA decode, step t,
+ *     one layer): the G new key/value vectors of the step are written into the cache at row t,
+ *     then every query head h looks up its group g(h) = ceil(h / (H/G)) (1-indexed), scores
+ *     q_h against K_cache[:t+1, g] scaled by 1/sqrt(d_k), takes a softmax over those t+1
+ *     scores and returns the weighted sum of V_cache[:t+1, g].
+ *   - Same page, Algorithm 1 (MHA decode): the same step with one key/value head per query
+ *     head; G = H reproduces it.
+ *   - Lesson "r-tf2-gqa" (ttlab.hopto.org), sections on how the heads are grouped and what
+ *     shrinks: query heads are grouped in contiguous blocks, and a grouped layer is run by
+ *     repeating each key/value head for the query heads of its block and then running
+ *     ordinary per-head attention ("expand then attend").
+ *
+ * The oracle follows that second form literally: expand_kv() materialises the repeated
+ * key/value heads of one sequence, attend_one_head() is textbook single-head softmax attention.
+ * Everything is float64, loops run in a fixed order, and there is no blocking, fusion or
+ * online rescaling.  With 0-indexed heads the contiguous-block map is g(h) = floor(h / r),
+ * r = H_q / H_kv, which is the 1-indexed ceil(h / (H/G)) of Algorithm 2 shifted by one.
+ *
+ * Readings where the pages leave a step open:
+ *   - Algorithm 2 appends before it attends, so the new token attends to itself: a sequence
+ *     whose cache held s rows before the step attends over n = s + 1 rows.
+ *   - A sequence with n = 0 rows has no softmax; its output is defined here as zeros.
+ *   - An append into a full cache (s >= L_max) is refused: the row is skipped, the length is
+ *     left alone and bit 1 of *status is set.  A length outside [0, L_max] at decode time
+ *     sets bit 2 and that sequence's output is zeros.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_APPEND_OVERFLOW 1
+#define ORACLE_SEQLEN_RANGE 2
+
+/* Algorithm 2, lines that write the new K/V row: K_cache[t, g, :] = k_g_new (and V alike),
+ * for every key/value head g of every sequence b, at t = the sequence's current length;
+ * the length then grows by one. */
+void oracle_kv_append(const double *k_new, const double *v_new, double *k_cache, double *v_cache,
+                      int32_t *seq_lens, int B, int H_kv, int d, int L_max, int32_t *status) {
+    for (int b = 0; b < B; ++b) {
+        int32_t t = seq_lens[b];
+        if (t < 0 || t >= L_max) {
+            if (status) *status |= ORACLE_APPEND_OVERFLOW;
+            continue;
+        }
+        for (int g = 0; g < H_kv; ++g) {
+            for (int i = 0; i < d; ++i) {
+                size_t src = ((size_t)b * H_kv + g) * d + i;
+                size_t dst = (((size_t)b * L_max + t) * H_kv + g) * d + i;
+                k_cache[dst] = k_new[src];
+                v_cache[dst] = v_new[src];
+            }
+        }
+        seq_lens[b] = t + 1;
+    }
+}
+
+/* "Expand then attend", first half: for one sequence, repeat key/value head floor(h / r)
+ * for query head h.  cache_b is [L_max][H_kv][d]; out is [n][H_q][d]. */
+void oracle_expand_kv(const double *cache_b, int n, int H_q, int H_kv, int d, double *out) {
+    int r = H_q / H_kv;
+    for (int t = 0; t < n; ++t) {
+        for (int h = 0; h < H_q; ++h) {
+            int g = h / r;
+            for (int i = 0; i < d; ++i) {
+                out[((size_t)t * H_q + h) * d + i] = cache_b[((size_t)t * H_kv + g) * d + i];
+            }
+        }
+    }
+}
+
+/* Textbook single-head attention for one query vector, as in Algorithm 1/2 of
+ * "GQA 阅读笔记": scores_t = scale * <q, K_t>, attn = softmax(scores), out = sum_t attn_t V_t.
+ * K and V rows are `row_stride` doubles apart.  The softmax subtracts the largest score before
+ * exponentiating (an exact identity that keeps exp() finite).  `weights` receives the n
+ * softmax weights when it is not NULL. */
+void oracle_attend_one_head(const double *q, const double *K, const double *V, int n, int d,
+                            size_t row_stride, double scale, double *out, double *weights) {
+    for (int i = 0; i < d; ++i) out[i] = 0.0;
+    if (n <= 0) return;
+    double *s = (double *)malloc(sizeof(double) * (size_t)n);
+    double m = -INFINITY;
+    for (int t = 0; t < n; ++t) {
+        double acc = 0.0;
+        for (int i = 0; i < d; ++i) acc += q[i] * K[(size_t)t * row_stride + i];
+        s[t] = scale * acc;
+        if (s[t] > m) m = s[t];
+    }
+    double z = 0.0;
+    for (int t = 0; t < n; ++t) {
+        s[t] = exp(s[t] - m);
+        z += s[t];
+    }
+    for (int t = 0; t < n; ++t) {
+        double w = s[t] / z;
+        if (weights) weights[t] = w;
+        for (int i = 0; i < d; ++i) out[i] += w * V[(size_t)t * row_stride + i];
+    }
+    free(s);
+}
+
+/* One decode step's attention for every sequence and query head.
+ *   q       [B][H_q][d]
+ *   k_cache [B][L_max][H_kv][d], v_cache alike
+ *   seq_lens[B]: rows each sequence attends over (already counting this step's appended row)
+ *   out     [B][H_q][d]
+ * Returns 0, or -1 when H_q is not a multiple of H_kv (the lesson page "r-tf2-gqa" requires
+ * h to be divisible by g) or a size is not positive.  nthreads <= 0 uses the OpenMP default. */
+int oracle_gqa_decode(const double *q, const double *k_cache, const double *v_cache,
+                      const int32_t *seq_lens, int B, int H_q, int H_kv, int d, int L_max,
+                      double scale, double *out, int nthreads, int32_t *status) {
+    if (B < 0 || H_q <= 0 || H_kv <= 0 || d <= 0 || L_max < 0 || H_q % H_kv != 0) return -1;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+    for (int b = 0; b < B; ++b) {
+        int n = seq_lens[b];
+        if (n < 0 || n > L_max) {
+            if (status) *status |= ORACLE_SEQLEN_RANGE;
+            n = 0;
+        }
+        size_t per_seq = (size_t)L_max * H_kv * d;
+        size_t expanded = (size_t)n * H_q * d;
+        double *Kx = (double *)malloc(sizeof(double) * (expanded ? expanded : 1));
+        double *Vx = (double *)malloc(sizeof(double) * (expanded ? expanded : 1));
+        oracle_expand_kv(k_cache + (size_t)b * per_seq, n, H_q, H_kv, d, Kx);
+        oracle_expand_kv(v_cache + (size_t)b * per_seq, n, H_q, H_kv, d, Vx);
+#pragma omp parallel for schedule(static)
+        for (int h = 0; h < H_q; ++h) {
+            oracle_attend_one_head(q + ((size_t)b * H_q + h) * d, Kx + (size_t)h * d,
+                                   Vx + (size_t)h * d, n, d, (size_t)H_q * d, scale,
+                                   out + ((size_t)b * H_q + h) * d, NULL);
+        }
+        free(Kx);
+        free(Vx);
+    }
+    return 0;
+}
+
+/* Number of threads the OpenMP runtime will use for the next parallel region. */
+int oracle_max_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

@@ -1,0 +1,46 @@
+"""Plant plausible mistakes in copies of the oracle and check that some pin catches each.
+
+Each mutant is one textual edit of oracle/gqa_oracle.c (a wrong head->group map, a dropped
+scale, an off-by-one length, a missing normalisation, a swapped operand, a wrong sign, a
+misplaced append), compiled to a temporary library on the CPU.  The committed oracle is never
+modified.
+"""
+import os
+
+import pytest
+
+import oracle as oracle_mod
+import oracle_pins
+
+SRC = os.path.join(os.path.dirname(oracle_mod.__file__), "gqa_oracle.c")
+
+MUTANTS = {
+    "group_map_modulo": ("int g = h / r;", "int g = h % H_kv;"),
+    "dropped_scale": ("s[t] = scale * acc;", "s[t] = acc;"),
+    "skips_appended_row": ("int n = seq_lens[b];", "int n = seq_lens[b] - 1;"),
+    "unnormalised": ("double w = s[t] / z;", "double w = s[t];"),
+    "weights_keys_not_values": ("out[i] += w * V[(size_t)t * row_stride + i];",
+                                "out[i] += w * K[(size_t)t * row_stride + i];"),
+    "scores_against_values": ("acc += q[i] * K[(size_t)t * row_stride + i];",
+                              "acc += q[i] * V[(size_t)t * row_stride + i];"),
+    "wrong_sign": ("s[t] = exp(s[t] - m);", "s[t] = exp(m - s[t]);"),
+    "no_max": ("if (s[t] > m) m = s[t];", "(void)0;"),
+    "append_off_by_one": ("size_t dst = (((size_t)b * L_max + t) * H_kv + g) * d + i;",
+                          "size_t dst = (((size_t)b * L_max + (t ? t - 1 : 0)) * H_kv + g) * d + i;"),
+    "append_no_length_update": ("seq_lens[b] = t + 1;", "seq_lens[b] = t;"),
+    "expand_wrong_head": ("out[((size_t)t * H_q + h) * d + i] = cache_b[((size_t)t * H_kv + g) * d + i];",
+                          "out[((size_t)t * H_q + h) * d + i] = cache_b[((size_t)t * H_kv + (H_kv - 1 - g)) * d + i];"),
+    "no_divisibility_check": ("H_q % H_kv != 0) return -1;", "0) return -1;"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(tmp_path, name):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
+    mutated = tmp_path / "mutant.c"
+    mutated.write_text(src.replace(old, new))
+    lib = oracle_mod.build(str(mutated), str(tmp_path / "libmutant.so"))
+    failed = oracle_pins.failing_pins(oracle_mod.Oracle(lib))
+    assert failed, f"mutant {name} passed every pin"
