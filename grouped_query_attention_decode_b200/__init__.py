@@ -1,0 +1,146 @@
+"""Python binding of libgqa: one grouped-query-attention decode step on B200.
+
+This module only marshals arguments: it takes torch tensors (device memory the caller
+allocated), passes their pointers, sizes and the current CUDA stream to the C ABI declared in
+``include/gqa.h``, and turns error codes into exceptions.  Every step of the computation runs in
+the library's CUDA kernels; there is no fallback.  If ``libgqa.so`` has not been built, importing
+the binding's functions raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgqa.so")
+
+DTYPE_F32 = 0
+DTYPE_BF16 = 1
+_DTYPES = {torch.float32: DTYPE_F32, torch.bfloat16: DTYPE_BF16}
+
+# status bits written by the kernels (include/gqa.h)
+STATUS_APPEND_OVERFLOW = 1
+STATUS_SEQLEN_RANGE = 2
+STATUS_WAIT_TIMEOUT = 4
+STATUS_INTERNAL = 8
+
+# C-ABI symbols declared in include/gqa.h
+EXPORTED = ("gqa_kv_append", "gqa_decode_workspace_size", "gqa_decode", "gqa_status_string",
+            "gqa_set_wait_timeout_ns", "gqa_profile_events")
+
+
+class GQAError(RuntimeError):
+    """A libgqa call returned a negative GQA_ERR_* code."""
+
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"libgqa error {code}: {msg}")
+        self.code = code
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libgqa.so (once).  Raises OSError when it is missing: build it first with
+    ``python -m grouped_query_attention_decode_b200.build``."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise OSError(f"{path} not found; build it with `python -m grouped_query_attention_decode_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, i32p = ctypes.c_void_p, ctypes.c_void_p
+    c_int, c_size = ctypes.c_int, ctypes.c_size_t
+    lib.gqa_kv_append.argtypes = [vp, vp, vp, vp, i32p, c_int, c_int, c_int, c_int, c_int, i32p, vp]
+    lib.gqa_kv_append.restype = c_int
+    lib.gqa_decode_workspace_size.argtypes = [c_int, c_int, c_int, c_int, c_int]
+    lib.gqa_decode_workspace_size.restype = c_size
+    lib.gqa_decode.argtypes = [vp, vp, vp, i32p, c_int, c_int, c_int, c_int, c_int,
+                               ctypes.c_float, c_int, vp, vp, c_size, i32p, vp]
+    lib.gqa_decode.restype = c_int
+    lib.gqa_status_string.argtypes = [c_int]
+    lib.gqa_status_string.restype = ctypes.c_char_p
+    lib.gqa_set_wait_timeout_ns.argtypes = [ctypes.c_ulonglong]
+    lib.gqa_set_wait_timeout_ns.restype = c_int
+    lib.gqa_profile_events.argtypes = [vp, vp]
+    lib.gqa_profile_events.restype = c_int
+    _lib = lib
+    return lib
+
+
+def status_string(code: int) -> str:
+    return load_library().gqa_status_string(int(code)).decode()
+
+
+def _check(rc: int):
+    if rc != 0:
+        raise GQAError(rc, status_string(rc))
+
+
+def _ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("libgqa needs contiguous tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype not in _DTYPES:
+        raise ValueError(f"unsupported dtype {t.dtype}")
+    return _DTYPES[t.dtype]
+
+
+def kv_append(k_new, v_new, k_cache, v_cache, seq_lens, status=None, stream=None) -> None:
+    """gqa_kv_append: k_cache[b, seq_lens[b]] = k_new[b] (and V), then seq_lens[b] += 1."""
+    B, L_max, H_kv, d = k_cache.shape
+    _check(load_library().gqa_kv_append(
+        _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens),
+        B, H_kv, d, L_max, _dtype(k_cache), _ptr(status), _stream(stream)))
+
+
+def workspace_size(B: int, H_q: int, H_kv: int, d: int, dtype: torch.dtype) -> int:
+    """Bytes of workspace gqa_decode needs on the current device."""
+    return int(load_library().gqa_decode_workspace_size(B, H_q, H_kv, d, _DTYPES[dtype]))
+
+
+def alloc_workspace(B: int, H_q: int, H_kv: int, d: int, dtype: torch.dtype, device=None):
+    n = workspace_size(B, H_q, H_kv, d, dtype)
+    if n == 0:
+        raise GQAError(-9, "no usable sm_100 device is current, or invalid sizes")
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def decode(q, k_cache, v_cache, seq_lens, scale: float, out=None, workspace=None, status=None,
+           stream=None) -> torch.Tensor:
+    """gqa_decode: attention of one decode step.  Returns ``out`` [B, H_q, d] float32."""
+    B, H_q, d = q.shape
+    _, L_max, H_kv, _ = k_cache.shape
+    if out is None:
+        out = torch.empty((B, H_q, d), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(B, H_q, H_kv, d, k_cache.dtype, device=q.device)
+    _check(load_library().gqa_decode(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens), B, H_q, H_kv, d, L_max,
+        float(scale), _dtype(k_cache), _ptr(out), _ptr(workspace), workspace.numel(),
+        _ptr(status), _stream(stream)))
+    return out
+
+
+def set_wait_timeout_ns(ns: int) -> None:
+    """Time limit of the decode kernels' internal waits (0 restores the 2 s default)."""
+    _check(load_library().gqa_set_wait_timeout_ns(int(ns)))
+
+
+def profile_events(before_split=None, after_split=None) -> None:
+    """Record these torch.cuda.Events around every later split-KV kernel (None, None stops)."""
+    a = ctypes.c_void_p(before_split.cuda_event) if before_split is not None else None
+    b = ctypes.c_void_p(after_split.cuda_event) if after_split is not None else None
+    _check(load_library().gqa_profile_events(a, b))

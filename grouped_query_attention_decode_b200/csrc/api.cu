@@ -1,0 +1,248 @@
+// C-ABI entry points of libgqa (declared and documented in include/gqa.h): argument checks,
+// workspace sizing, TMA descriptor encoding and kernel launches.  No device memory is
+// allocated here.
+#include <cuda.h>
+#include <cuda_runtime_api.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "gqa.h"
+#include "launch.h"
+#include "schedule.cuh"
+
+namespace gqa {
+namespace {
+
+constexpr unsigned long long kDefaultWaitNs = 2000000000ull;
+std::atomic<unsigned long long> g_wait_ns{kDefaultWaitNs};
+std::atomic<cudaEvent_t> g_ev_before{nullptr};
+std::atomic<cudaEvent_t> g_ev_after{nullptr};
+
+constexpr int kMaxDevices = 64;
+int g_sm_count[kMaxDevices] = {};
+std::mutex g_mu;
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// SM count of the current device, or <= 0 when there is none (or it is not sm_100).
+int current_sm_count(int *dev_out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return 0;
+    }
+    *dev_out = dev;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_sm_count[dev] == 0) {
+        int sms = 0, major = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return 0;
+        }
+        g_sm_count[dev] = (major == 10) ? sms : -1;
+    }
+    return g_sm_count[dev];
+}
+
+struct Geometry {
+    int r, RB, HB, UB;
+    long long units, slots, slot_floats, hdr_floats;
+    size_t bytes;
+};
+
+Geometry geometry(int B, int H_q, int H_kv, int d, int G) {
+    Geometry g;
+    g.r = H_q / H_kv;
+    g.RB = g.r < 64 ? g.r : 64;
+    g.HB = (g.r + g.RB - 1) / g.RB;
+    g.UB = H_kv * g.HB;
+    g.units = static_cast<long long>(B) * g.UB;
+    g.slots = G + g.units - 1;
+    g.slot_floats = static_cast<long long>(g.RB) * (d + 2);
+    g.hdr_floats = ((static_cast<long long>(B) + 1) * 8 + 255) / 256 * 64;  // 256-byte multiple
+    g.bytes = static_cast<size_t>((g.hdr_floats + g.slots * g.slot_floats) * 4 + 255) / 256 * 256;
+    return g;
+}
+
+int check_shape(int B, int H_q, int H_kv, int d, int L_max, gqa_dtype_t dtype) {
+    if (dtype != GQA_DTYPE_F32 && dtype != GQA_DTYPE_BF16) return GQA_ERR_UNSUPPORTED_DTYPE;
+    if (B <= 0 || H_q <= 0 || H_kv <= 0 || L_max <= 0) return GQA_ERR_SHAPE;
+    if (H_q % H_kv != 0) return GQA_ERR_HEADS_NOT_DIVISIBLE;
+    if (d != 64 && d != 128) return GQA_ERR_UNSUPPORTED_DIM;
+    // Index arithmetic in the kernels: rows of q and tiles per launch stay well inside int32.
+    if (static_cast<long long>(B) * H_q > (1ll << 30) || static_cast<long long>(B) * H_kv > (1ll << 30))
+        return GQA_ERR_SHAPE;
+    return GQA_OK;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                             &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+        else
+            cudaGetLastError();
+    });
+    return fn;
+}
+
+bool encode_cache_map(CUtensorMap *m, const void *base, int B, int H_kv, int d, int L_max, int rows) {
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H_kv),
+                                static_cast<cuuint64_t>(L_max), static_cast<cuuint64_t>(B)};
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 2,
+                                   static_cast<cuuint64_t>(H_kv) * d * 2,
+                                   static_cast<cuuint64_t>(L_max) * H_kv * d * 2};
+    const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(rows), 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims,
+                       strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                       CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool encode_q_map(CUtensorMap *m, const void *q, int B, int H_q, int d, int rp) {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(B) * H_q};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
+    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(rp)};
+    const cuuint32_t estr[2] = {1, 1};
+    return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(q), dims,
+                       strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                       CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+}  // namespace gqa
+
+using namespace gqa;
+
+extern "C" int gqa_kv_append(const void *k_new, const void *v_new, void *k_cache, void *v_cache,
+                             int32_t *seq_lens, int B, int H_kv, int d, int L_max,
+                             gqa_dtype_t dtype, int32_t *status, cudaStream_t stream) {
+    if (!k_new || !v_new || !k_cache || !v_cache || !seq_lens) return GQA_ERR_NULL;
+    if (dtype != GQA_DTYPE_F32 && dtype != GQA_DTYPE_BF16) return GQA_ERR_UNSUPPORTED_DTYPE;
+    if (B <= 0 || H_kv <= 0 || L_max <= 0 || static_cast<long long>(B) * H_kv > (1ll << 30))
+        return GQA_ERR_SHAPE;
+    if (d != 64 && d != 128) return GQA_ERR_UNSUPPORTED_DIM;
+    if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(k_cache, 16) ||
+        !aligned(v_cache, 16) || !aligned(seq_lens, 4) || (status && !aligned(status, 4)))
+        return GQA_ERR_ALIGNMENT;
+    int dev = 0;
+    if (current_sm_count(&dev) <= 0) return GQA_ERR_NO_DEVICE;
+    const int row_bytes = d * (dtype == GQA_DTYPE_BF16 ? 2 : 4);
+    return launch_append(k_new, v_new, k_cache, v_cache, seq_lens, B, H_kv, row_bytes, L_max,
+                         status, stream);
+}
+
+extern "C" size_t gqa_decode_workspace_size(int B, int H_q, int H_kv, int d, gqa_dtype_t dtype) {
+    if (check_shape(B, H_q, H_kv, d, 1, dtype) != GQA_OK) return 0;
+    int dev = 0;
+    const int sms = current_sm_count(&dev);
+    if (sms <= 0) return 0;
+    return geometry(B, H_q, H_kv, d, sms).bytes;
+}
+
+extern "C" int gqa_decode(const void *q, const void *k_cache, const void *v_cache,
+                          const int32_t *seq_lens, int B, int H_q, int H_kv, int d, int L_max,
+                          float scale, gqa_dtype_t dtype, float *out, void *workspace,
+                          size_t workspace_bytes, int32_t *status, cudaStream_t stream) {
+    if (!q || !k_cache || !v_cache || !seq_lens || !out) return GQA_ERR_NULL;
+    const int rc = check_shape(B, H_q, H_kv, d, L_max, dtype);
+    if (rc != GQA_OK) return rc;
+    if (!workspace) return GQA_ERR_WORKSPACE;
+    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16) ||
+        !aligned(seq_lens, 4) || !aligned(workspace, 256) || (status && !aligned(status, 4)))
+        return GQA_ERR_ALIGNMENT;
+    if (!std::isfinite(scale)) return GQA_ERR_SHAPE;
+    int dev = 0;
+    const int sms = current_sm_count(&dev);
+    if (sms <= 0) return GQA_ERR_NO_DEVICE;
+    const Geometry g = geometry(B, H_q, H_kv, d, sms);
+    if (workspace_bytes < g.bytes) return GQA_ERR_WORKSPACE;
+
+    DecodeParams p;
+    p.seq_lens = seq_lens;
+    p.out = out;
+    p.ws = static_cast<float *>(workspace);
+    p.status = status;
+    p.B = B;
+    p.H_q = H_q;
+    p.H_kv = H_kv;
+    p.d = d;
+    p.L_max = L_max;
+    p.r = g.r;
+    p.RB = g.RB;
+    p.HB = g.HB;
+    p.UB = g.UB;
+    p.T = dtype == GQA_DTYPE_BF16 ? 128 : 64;
+    p.G = sms;
+    p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    p.wait_ns = g_wait_ns.load();
+    p.slot_floats = g.slot_floats;
+    p.hdr_floats = g.hdr_floats;
+
+    cudaEvent_t ev0 = g_ev_before.load(), ev1 = g_ev_after.load();
+    const bool profile = ev0 != nullptr && ev1 != nullptr;
+    int res;
+    if (dtype == GQA_DTYPE_BF16) {
+        const int rp = g.RB <= 16 ? 16 : (g.RB <= 32 ? 32 : 64);
+        if (encode_fn() == nullptr) return GQA_ERR_CUDA;
+        TmaMaps maps;
+        if (!encode_q_map(&maps.q, q, B, H_q, d, rp) ||
+            !encode_cache_map(&maps.k, k_cache, B, H_kv, d, L_max, 128) ||
+            !encode_cache_map(&maps.k8, k_cache, B, H_kv, d, L_max, 8) ||
+            !encode_cache_map(&maps.v, v_cache, B, H_kv, d, L_max, 128) ||
+            !encode_cache_map(&maps.v8, v_cache, B, H_kv, d, L_max, 8))
+            return GQA_ERR_SHAPE;
+        if (profile && cudaEventRecord(ev0, stream) != cudaSuccess) return GQA_ERR_CUDA;
+        res = launch_split_tc(maps, p, rp, stream);
+    } else {
+        if (profile && cudaEventRecord(ev0, stream) != cudaSuccess) return GQA_ERR_CUDA;
+        res = launch_split_f32(p, static_cast<const float *>(q), static_cast<const float *>(k_cache),
+                               static_cast<const float *>(v_cache), stream);
+    }
+    if (res != GQA_OK) return res;
+    if (profile && cudaEventRecord(ev1, stream) != cudaSuccess) return GQA_ERR_CUDA;
+    return launch_combine(p, stream);
+}
+
+extern "C" const char *gqa_status_string(int code) {
+    switch (code) {
+        case GQA_OK: return "ok";
+        case GQA_ERR_NULL: return "a required pointer is NULL";
+        case GQA_ERR_SHAPE: return "a size is not positive, too large, or not representable";
+        case GQA_ERR_HEADS_NOT_DIVISIBLE: return "H_q is not a multiple of H_kv";
+        case GQA_ERR_UNSUPPORTED_DIM: return "head dimension d must be 64 or 128";
+        case GQA_ERR_UNSUPPORTED_DTYPE: return "unsupported element type";
+        case GQA_ERR_ALIGNMENT: return "a pointer is not aligned as required";
+        case GQA_ERR_WORKSPACE: return "workspace is NULL or too small";
+        case GQA_ERR_CUDA: return "a CUDA runtime call failed";
+        case GQA_ERR_NO_DEVICE: return "no usable sm_100 device is current";
+        default: return "unknown status code";
+    }
+}
+
+extern "C" int gqa_set_wait_timeout_ns(unsigned long long ns) {
+    g_wait_ns.store(ns == 0 ? kDefaultWaitNs : ns);
+    return GQA_OK;
+}
+
+extern "C" int gqa_profile_events(cudaEvent_t before_split, cudaEvent_t after_split) {
+    g_ev_before.store(before_split);
+    g_ev_after.store(after_split);
+    return GQA_OK;
+}

@@ -1,0 +1,81 @@
+// Log-sum-exp combine of split-KV partial results.
+//
+// A piece c of a unit holds, per query head, the unnormalised sum o_c = sum_t 2^(x_t - m_c) v_t,
+// its reference m_c (log2 units) and l_c = sum_t 2^(x_t - m_c).  Because softmax is a ratio of
+// sums of exponentials, the pieces merge exactly:
+//     M = max_c m_c,   out = sum_c 2^(m_c - M) o_c / sum_c 2^(m_c - M) l_c.
+// The pages state the blockwise idea (split the sequence into blocks, compute each block
+// independently, then merge: "GQA注意力机制", section 4.2); the merge rule is the softmax
+// algebra above.  Units covered by a single piece were finished by the split kernel and are
+// skipped; units with no rows get zeros.
+#include <cstdint>
+
+#include "device.cuh"
+#include "gqa.h"
+#include "launch.h"
+#include "schedule.cuh"
+
+namespace gqa {
+
+__global__ void __launch_bounds__(256) combine_kernel(const DecodeParams p) {
+    grid_dependency_wait();
+    const int u = blockIdx.x;
+    const int b = u / p.UB;
+    const int k = u - b * p.UB;
+    const int kvh = k / p.HB;
+    const int hb = k - kvh * p.HB;
+    const int nh = min(p.RB, p.r - hb * p.RB);
+    const int h0 = kvh * p.r + hb * p.RB;
+    const int d = p.d;
+    float *o = p.out + (static_cast<long long>(b) * p.H_q + h0) * d;
+    const long long *hdr = reinterpret_cast<const long long *>(p.ws);
+    const int n = valid_len(p.seq_lens[b], p.L_max);
+    const int nt = tiles_of(n, p.T);
+    if (nt == 0) {
+        for (int idx = threadIdx.x; idx < nh * d; idx += blockDim.x) o[idx] = 0.f;
+        return;
+    }
+    const long long total = hdr[p.B];
+    const long long uoff = hdr[b] + static_cast<long long>(k) * nt;
+    const long long i0 = cta_of_tile(uoff, total, p.G);
+    const long long i1 = cta_of_tile(uoff + nt - 1, total, p.G);
+    if (i0 == i1) return;
+    const float *slots = p.ws + p.hdr_floats;
+    for (int idx = threadIdx.x; idx < nh * d; idx += blockDim.x) {
+        const int h = idx / d;
+        float M = -INFINITY;
+        for (long long i = i0; i <= i1; ++i) {
+            if (cta_range_begin(i, total, p.G) == cta_range_begin(i + 1, total, p.G)) continue;
+            const float *s = slots + (i + u) * p.slot_floats;
+            M = fmaxf(M, s[nh * d + h]);
+        }
+        float num = 0.f, den = 0.f;
+        for (long long i = i0; i <= i1; ++i) {
+            if (cta_range_begin(i, total, p.G) == cta_range_begin(i + 1, total, p.G)) continue;
+            const float *s = slots + (i + u) * p.slot_floats;
+            const float wgt = ex2_approx(s[nh * d + h] - M);
+            num = fmaf(wgt, s[idx], num);
+            den = fmaf(wgt, s[nh * d + nh + h], den);
+        }
+        o[idx] = num / den;
+    }
+}
+
+int launch_combine(const DecodeParams &p, cudaStream_t stream) {
+    const long long units = static_cast<long long>(p.B) * p.UB;
+    if (units == 0) return GQA_OK;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(units));
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, combine_kernel, p) != cudaSuccess) return GQA_ERR_CUDA;
+    return GQA_OK;
+}
+
+}  // namespace gqa

@@ -1,0 +1,27 @@
+// Host-side declarations shared by the kernel files and the C-ABI entry points.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime_api.h>
+
+#include <cstdint>
+
+namespace gqa {
+
+struct DecodeParams;
+
+// TMA descriptors of one bf16 decode call: q as [B*H_q rows][d], the caches as
+// (d, H_kv, L_max, B) with 128-row and 8-row boxes of 64 columns, all with 128-byte swizzle.
+struct TmaMaps {
+    CUtensorMap q, k, k8, v, v8;
+};
+
+int launch_split_tc(const TmaMaps &maps, const DecodeParams &p, int rp, cudaStream_t stream);
+int launch_split_f32(const DecodeParams &p, const float *q, const float *kc, const float *vc,
+                     cudaStream_t stream);
+int launch_combine(const DecodeParams &p, cudaStream_t stream);
+int launch_append(const void *k_new, const void *v_new, void *k_cache, void *v_cache,
+                  int32_t *seq_lens, int B, int H_kv, int row_bytes, int L_max, int32_t *status,
+                  cudaStream_t stream);
+
+}  // namespace gqa

@@ -1,0 +1,184 @@
+// Work partition shared by the split-KV kernels and the combine kernel.
+//
+// The decode work is cut into tiles of T cached rows.  A "unit" is one (sequence b, key/value
+// head j, block of up to 64 query heads of j's group); a unit has ceil(n_b / T) tiles.  Units
+// are ordered b-major, and the tiles of all units form one line of `total` tiles.  The split
+// kernel runs G persistent CTAs and CTA i takes the contiguous tile range
+//     [floor(i * total / G), floor((i + 1) * total / G)),
+// so every CTA streams the same number of tiles (to within one) whatever the length mix.  A
+// CTA range may cut a unit; each (CTA, unit) piece produces a partial result in workspace
+// slot (CTA index + unit index), which is unique because both indices grow along the line.
+// A unit covered by a single piece is finished by that CTA; the others are merged by the
+// combine kernel.  Every kernel derives the same partition from seq_lens on the device, so
+// the host never needs the lengths.
+#pragma once
+
+#include <cstdint>
+
+#include "device.cuh"
+#include "gqa.h"
+
+namespace gqa {
+
+struct DecodeParams {
+    const int32_t *seq_lens;  // [B] rows attended per sequence
+    float *out;               // [B][H_q][d]
+    float *ws;                // workspace: int64 header, then partial slots
+    int32_t *status;          // device status word or nullptr
+    int B, H_q, H_kv, d, L_max;
+    int r;     // query heads per key/value head
+    int RB;    // query heads per unit (<= 64)
+    int HB;    // units per key/value head = ceil(r / RB)
+    int UB;    // units per sequence = H_kv * HB
+    int T;     // cached rows per tile
+    int G;     // CTAs of the split kernel
+    float scale_log2;                 // softmax scale * log2(e)
+    unsigned long long wait_ns;       // bound of every pipeline wait
+    long long slot_floats;            // RB * (d + 2)
+    long long hdr_floats;             // header length in floats (int64 offsets [B + 1])
+};
+
+__device__ __forceinline__ int valid_len(int n, int L_max) {
+    return (n < 0 || n > L_max) ? 0 : n;
+}
+
+__device__ __forceinline__ int tiles_of(int n, int T) { return (n + T - 1) / T; }
+
+__device__ __forceinline__ long long cta_range_begin(long long i, long long total, long long G) {
+    return i * total / G;
+}
+
+// The CTA whose range holds tile t (the largest i with begin(i) <= t).
+__device__ __forceinline__ long long cta_of_tile(long long t, long long total, long long G) {
+    return ((t + 1) * G - 1) / total;
+}
+
+__device__ __forceinline__ long long warp_incl_scan(long long v, int lane) {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        long long u = __shfl_up_sync(kFullMask, v, o);
+        if (lane >= o) v += u;
+    }
+    return v;
+}
+
+struct CtaRange {
+    long long begin, end, total;
+    int b0;          // first sequence with a tile in [begin, end) (valid when begin < end)
+    long long off0;  // first tile of sequence b0 on the line
+};
+
+// Whole warp: total tiles, this CTA's range and where it starts.  When `hdr` is not null the
+// warp also stores the exclusive prefix of tiles per sequence (hdr[b], b <= B; hdr[B] = total).
+// When `flag_range` is set, lengths outside [0, L_max] set GQA_STATUS_SEQLEN_RANGE.
+__device__ inline CtaRange locate_cta_range(const DecodeParams &p, int cta, int lane, long long *hdr,
+                                     bool flag_range) {
+    long long run = 0;
+    for (int base = 0; base < p.B; base += 32) {
+        const int b = base + lane;
+        int n = 0;
+        if (b < p.B) {
+            const int raw = p.seq_lens[b];
+            n = valid_len(raw, p.L_max);
+            if (flag_range && n != raw && p.status != nullptr) atomicOr(p.status, GQA_STATUS_SEQLEN_RANGE);
+        }
+        const long long v = static_cast<long long>(tiles_of(n, p.T)) * p.UB;
+        const long long incl = warp_incl_scan(v, lane);
+        if (hdr != nullptr && b < p.B) hdr[b] = run + incl - v;
+        run += __shfl_sync(kFullMask, incl, 31);
+    }
+    CtaRange cr;
+    cr.total = run;
+    if (hdr != nullptr && lane == 0) hdr[p.B] = run;
+    cr.begin = cta_range_begin(cta, run, p.G);
+    cr.end = cta_range_begin(cta + 1, run, p.G);
+    cr.b0 = 0;
+    cr.off0 = 0;
+    if (cr.begin >= cr.end) return cr;
+    long long off = 0;
+    for (int base = 0; base < p.B; base += 32) {
+        const int b = base + lane;
+        const int n = b < p.B ? valid_len(p.seq_lens[b], p.L_max) : 0;
+        const long long v = static_cast<long long>(tiles_of(n, p.T)) * p.UB;
+        const long long incl = warp_incl_scan(v, lane);
+        const long long excl = incl - v;
+        const bool hit = v > 0 && off + excl <= cr.begin && cr.begin < off + incl;
+        const uint32_t m = __ballot_sync(kFullMask, hit);
+        if (m != 0) {
+            const int l = __ffs(m) - 1;
+            cr.b0 = base + l;
+            cr.off0 = off + __shfl_sync(kFullMask, excl, l);
+            return cr;
+        }
+        off += __shfl_sync(kFullMask, incl, 31);
+    }
+    return cr;  // unreachable when begin < total
+}
+
+// One CTA-range piece of one unit.
+struct Segment {
+    int b, kvh, hb;  // sequence, key/value head, block of query heads
+    int j0, len;     // first tile (within the unit) and number of tiles of the piece
+    int n;           // rows attended by sequence b
+    int unit;        // unit index b * UB + (kvh * HB + hb)
+    bool whole;      // the piece is the entire unit
+};
+
+// Walks the segments of one CTA range in order.  Each role of the CTA runs its own walker;
+// all of them see the same sequence of segments.
+struct SegmentWalker {
+    const int32_t *lens;
+    int B, UB, HB, L_max, T;
+    int b, n, nt;
+    long long off, t, end;
+
+    __device__ void init(const DecodeParams &p, const CtaRange &cr) {
+        lens = p.seq_lens;
+        B = p.B;
+        UB = p.UB;
+        HB = p.HB;
+        L_max = p.L_max;
+        T = p.T;
+        t = cr.begin;
+        end = cr.end;
+        b = cr.b0;
+        off = cr.off0;
+        if (t < end) {
+            n = valid_len(lens[b], L_max);
+            nt = tiles_of(n, T);
+        } else {
+            n = 0;
+            nt = 0;
+        }
+    }
+
+    __device__ bool next(Segment &s) {
+        if (t >= end) return false;
+        while (t >= off + static_cast<long long>(nt) * UB) {
+            off += static_cast<long long>(nt) * UB;
+            if (++b >= B) {  // cannot happen while t < total; never read past seq_lens[B-1]
+                t = end;
+                return false;
+            }
+            n = valid_len(lens[b], L_max);
+            nt = tiles_of(n, T);
+        }
+        const long long rel = t - off;
+        const int k = static_cast<int>(rel / nt);
+        const int j0 = static_cast<int>(rel - static_cast<long long>(k) * nt);
+        const long long left = end - t;
+        const int len = static_cast<int>(left < nt - j0 ? left : nt - j0);
+        s.b = b;
+        s.kvh = k / HB;
+        s.hb = k - s.kvh * HB;
+        s.j0 = j0;
+        s.len = len;
+        s.n = n;
+        s.unit = b * UB + k;
+        s.whole = (j0 == 0 && len == nt);
+        t += len;
+        return true;
+    }
+};
+
+}  // namespace gqa

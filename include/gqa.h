@@ -1,0 +1,155 @@
+/*
+ * libgqa: one grouped-query-attention (GQA) decode step on NVIDIA B200 (sm_100a).
+ *
+ * The operation is Algorithm 2 ("GQA 解码，第 t 步，单层") of the reading notes "GQA 阅读笔记"
+ * (zhongzhuzhou.org, section "GQA 架构"), split into the two calls below:
+ *
+ *   gqa_kv_append  the lines that write this step's key/value vectors into the cache
+ *                  (K_cache[t, g, :] = k_g_new, V_cache[t, g, :] = v_g_new, for every group g);
+ *   gqa_decode     the per-head lines: head h reads the cache of its group g(h), scores
+ *                  q_h . K_cache[:t+1, g]^T * scale, takes a softmax over those t+1 scores and
+ *                  returns the weighted sum of V_cache[:t+1, g].
+ *
+ * With H_q query heads and H_kv key/value heads (H_kv = G, the number of groups), query heads
+ * are grouped in contiguous blocks of r = H_q / H_kv: query head h (0-indexed) uses key/value
+ * head h / r.  That is the page's 1-indexed g(h) = ceil(h / (H/G)).  H_kv = H_q is multi-head
+ * attention (Algorithm 1 of the same page), H_kv = 1 is multi-query attention.  The lesson
+ * "r-tf2-gqa" (ttlab.hopto.org) requires H_q to be a multiple of H_kv; other shapes are
+ * rejected.
+ *
+ * Conventions shared by every call:
+ *   - All tensors are dense, row-major, with the last dimension contiguous:
+ *       q        [B][H_q][d]           k_new, v_new [B][H_kv][d]
+ *       k_cache  [B][L_max][H_kv][d]   v_cache      [B][L_max][H_kv][d]
+ *       out      [B][H_q][d]  float32 (always float32, whatever the input dtype)
+ *       seq_lens [B]          int32
+ *     Every pointer is a DEVICE pointer except where a comment says otherwise.
+ *   - d is 64 or 128.  q, k_new, v_new and the caches share one element type (gqa_dtype_t).
+ *   - Device pointers must be 16-byte aligned; `workspace` must be 256-byte aligned.
+ *   - The caller owns and allocates every buffer, including the decode workspace.  The
+ *     library allocates no device memory and keeps no per-call state.
+ *   - Calls are asynchronous on `stream` (0 = the legacy default stream) and never
+ *     synchronize the host.  Errors the host can see (a NULL pointer, a bad shape, a
+ *     misaligned pointer, a short workspace) return a negative GQA_ERR_* code before anything
+ *     is launched.  Errors only the device can see set bits in *status (GQA_STATUS_*, combined
+ *     with atomicOr; `status` may be NULL) and skip the offending work; kernels never trap.
+ *   - A non-zero return of GQA_ERR_CUDA means a CUDA runtime call failed; the CUDA error is
+ *     left for cudaGetLastError().
+ */
+#ifndef GQA_H
+#define GQA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Element type of q, k_new, v_new, k_cache and v_cache. */
+typedef enum {
+    GQA_DTYPE_F32 = 0,  /* IEEE float32; computed on CUDA cores in float32 */
+    GQA_DTYPE_BF16 = 1  /* bfloat16; products on tcgen05 tensor cores, float32 accumulation */
+} gqa_dtype_t;
+
+/* Return codes. */
+#define GQA_OK 0
+#define GQA_ERR_NULL (-1)                 /* a required pointer is NULL */
+#define GQA_ERR_SHAPE (-2)                /* a size is not positive or too large */
+#define GQA_ERR_HEADS_NOT_DIVISIBLE (-3)  /* H_q is not a multiple of H_kv */
+#define GQA_ERR_UNSUPPORTED_DIM (-4)      /* d is not 64 or 128 */
+#define GQA_ERR_UNSUPPORTED_DTYPE (-5)    /* dtype is not a gqa_dtype_t value */
+#define GQA_ERR_ALIGNMENT (-6)            /* a pointer is not aligned as required */
+#define GQA_ERR_WORKSPACE (-7)            /* workspace NULL or smaller than required */
+#define GQA_ERR_CUDA (-8)                 /* a CUDA runtime call failed */
+#define GQA_ERR_NO_DEVICE (-9)            /* no usable sm_100 device is current */
+
+/* Device-side status bits (OR-ed into *status). */
+#define GQA_STATUS_APPEND_OVERFLOW 1  /* gqa_kv_append: seq_lens[b] < 0 or >= L_max; row skipped */
+#define GQA_STATUS_SEQLEN_RANGE 2     /* gqa_decode: seq_lens[b] < 0 or > L_max; out[b] = 0 */
+#define GQA_STATUS_WAIT_TIMEOUT 4     /* gqa_decode: a pipeline wait ran past its time limit;
+                                         the affected outputs are not valid */
+#define GQA_STATUS_INTERNAL 8         /* gqa_decode: shared-memory base not 1024-byte aligned */
+
+/*
+ * gqa_kv_append: write this step's key and value vectors into the cache.
+ *
+ * Algorithm 2 of "GQA 阅读笔记", the lines that write the new rows (and Algorithm 1's for
+ * MHA): for every sequence b and key/value head j, with t = seq_lens[b] on entry,
+ *     k_cache[b][t][j][:] = k_new[b][j][:],  v_cache[b][t][j][:] = v_new[b][j][:],
+ * then seq_lens[b] = t + 1.  The copy is bit-exact.  A sequence with t < 0 or t >= L_max is
+ * left untouched (cache and length) and sets GQA_STATUS_APPEND_OVERFLOW.
+ *
+ *   k_new, v_new  [B][H_kv][d] device, read
+ *   k_cache, v_cache [B][L_max][H_kv][d] device, written at row t only
+ *   seq_lens      [B] int32 device, read and incremented
+ *   status        int32 device or NULL
+ * Returns GQA_OK or a GQA_ERR_* code.
+ */
+int gqa_kv_append(const void *k_new, const void *v_new, void *k_cache, void *v_cache,
+                  int32_t *seq_lens, int B, int H_kv, int d, int L_max, gqa_dtype_t dtype,
+                  int32_t *status, cudaStream_t stream);
+
+/*
+ * gqa_decode_workspace_size: bytes of device workspace gqa_decode needs for these sizes on
+ * the CURRENT device (the count depends on its number of SMs).  Returns 0 when the sizes are
+ * invalid or no device is current.
+ */
+size_t gqa_decode_workspace_size(int B, int H_q, int H_kv, int d, gqa_dtype_t dtype);
+
+/*
+ * gqa_decode: the attention of one decode step, for every sequence and query head.
+ *
+ * Algorithm 2 of "GQA 阅读笔记", the per-head lines; with n = seq_lens[b] (the number of
+ * cached rows, already counting this step's appended row) and r = H_q / H_kv:
+ *     out[b][h][:] = sum_{t<n} softmax_t( scale * q[b][h] . k_cache[b][t][h/r] )
+ *                    * v_cache[b][t][h/r][:]
+ * Cache rows at or beyond n are never read.  n = 0 gives out[b] = 0 (a softmax over no rows
+ * is undefined; zero is this library's convention).  n < 0 or n > L_max gives out[b] = 0
+ * and sets GQA_STATUS_SEQLEN_RANGE.  Each cached K/V row is read from memory once per group
+ * and serves all r query heads of the group.
+ *
+ *   q          [B][H_q][d] device, read
+ *   k_cache, v_cache [B][L_max][H_kv][d] device, read (rows < seq_lens[b] only)
+ *   seq_lens   [B] int32 device, read
+ *   scale      softmax scale, usually 1/sqrt(d)
+ *   out        [B][H_q][d] float32 device, written
+ *   workspace  device scratch of at least gqa_decode_workspace_size() bytes, 256-byte aligned;
+ *              owned by the caller, overwritten by every call.  Two gqa_decode calls that may
+ *              run at the same time must not share one workspace.
+ *   status     int32 device or NULL
+ * Launches two kernels on `stream` (a split-KV pass and a log-sum-exp combine).
+ * Returns GQA_OK or a GQA_ERR_* code.
+ */
+int gqa_decode(const void *q, const void *k_cache, const void *v_cache, const int32_t *seq_lens,
+               int B, int H_q, int H_kv, int d, int L_max, float scale, gqa_dtype_t dtype,
+               float *out, void *workspace, size_t workspace_bytes, int32_t *status,
+               cudaStream_t stream);
+
+/* gqa_status_string: a static, human-readable string for a GQA_OK / GQA_ERR_* code. */
+const char *gqa_status_string(int code);
+
+/*
+ * gqa_set_wait_timeout_ns: time limit of every bounded wait inside the decode kernels, for
+ * the calls launched after it (process-wide).  ns = 0 restores the default of 2 s.  A
+ * kernel whose wait runs out sets GQA_STATUS_WAIT_TIMEOUT, waits for its own copies and
+ * tensor-core work already in flight, frees its tensor memory and returns.  Tests use a
+ * tiny limit to exercise that path without faulting the GPU.  Returns GQA_OK.
+ */
+int gqa_set_wait_timeout_ns(unsigned long long ns);
+
+/*
+ * gqa_profile_events: measurement hook (process-wide).  When both events are non-NULL, every
+ * later gqa_decode records `before_split` on its stream just before the split-KV kernel and
+ * `after_split` just after it, so the caller can time that kernel alone with
+ * cudaEventElapsedTime.  Pass NULL, NULL to stop.  The caller owns the events.  Returns GQA_OK.
+ */
+int gqa_profile_events(cudaEvent_t before_split, cudaEvent_t after_split);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GQA_H */
