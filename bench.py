@@ -60,6 +60,15 @@ def dist_env():
     return rank, world, local
 
 
+def max_over_ranks(x: float, pg, device) -> float:
+    """Max of a per-rank number over all ranks (the whole job is as slow as its slowest rank)."""
+    if pg is None:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -239,11 +248,7 @@ def bench_ours(args, rank, world, local):
     split_ms = [a.elapsed_time(b) for a, b in pairs]
     assert int(status.item()) == 0, f"device status {int(status.item())}"
 
-    ms_step = t_ms / K
-    if pg is not None:
-        t = torch.tensor([ms_step], dtype=torch.float64, device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms_step = float(t.item())
+    ms_step = max_over_ranks(t_ms / K, pg, dev)
     value = ideal * world / (ms_step * 1e-3) / 1e9
 
     # End to end through the public API: every step copies its inputs (q, k_new, v_new) in
@@ -274,11 +279,7 @@ def bench_ours(args, rank, world, local):
         e2e_step(i, lens_big[i])
     b.record(stream)
     torch.cuda.synchronize()
-    e2e_step_ms = a.elapsed_time(b) / ke
-    if pg is not None:
-        t = torch.tensor([e2e_step_ms], dtype=torch.float64, device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        e2e_step_ms = float(t.item())
+    e2e_step_ms = max_over_ranks(a.elapsed_time(b) / ke, pg, dev)
     assert np.isfinite(hout.numpy()).all()
     assert int(status.item()) == 0, f"device status {int(status.item())}"
     Ke = ke
