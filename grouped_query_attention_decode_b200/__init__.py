@@ -28,7 +28,7 @@ STATUS_INTERNAL = 8
 
 # C-ABI symbols declared in include/gqa.h
 EXPORTED = ("gqa_kv_append", "gqa_decode_workspace_size", "gqa_decode", "gqa_status_string",
-            "gqa_set_wait_timeout_ns", "gqa_profile_events")
+            "gqa_set_wait_timeout_ns", "gqa_profile_events", "gqa_decode_noalloc")
 
 
 class GQAError(RuntimeError):
@@ -60,6 +60,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gqa_decode.argtypes = [vp, vp, vp, i32p, c_int, c_int, c_int, c_int, c_int,
                                ctypes.c_float, c_int, vp, vp, c_size, i32p, vp]
     lib.gqa_decode.restype = c_int
+    lib.gqa_decode_noalloc.argtypes = [vp, vp, vp, i32p, c_int, c_int, c_int, c_int, c_int,
+                                       ctypes.c_float, c_int, vp, i32p, vp]
+    lib.gqa_decode_noalloc.restype = c_int
     lib.gqa_status_string.argtypes = [c_int]
     lib.gqa_status_string.restype = ctypes.c_char_p
     lib.gqa_set_wait_timeout_ns.argtypes = [ctypes.c_ulonglong]
@@ -131,6 +134,21 @@ def decode(q, k_cache, v_cache, seq_lens, scale: float, out=None, workspace=None
         _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens), B, H_q, H_kv, d, L_max,
         float(scale), _dtype(k_cache), _ptr(out), _ptr(workspace), workspace.numel(),
         _ptr(status), _stream(stream)))
+    return out
+
+
+def decode_noalloc(q, k_cache, v_cache, seq_lens, scale: float, out=None, status=None,
+                   stream=None) -> torch.Tensor:
+    """gqa_decode_noalloc: like ``decode`` but with the library's own fixed scratch array
+    instead of a caller workspace (for callers that cannot allocate one).  Calls that may run
+    at the same time on the GPU must not overlap: they share that array."""
+    B, H_q, d = q.shape
+    _, L_max, H_kv, _ = k_cache.shape
+    if out is None:
+        out = torch.empty((B, H_q, d), dtype=torch.float32, device=q.device)
+    _check(load_library().gqa_decode_noalloc(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens), B, H_q, H_kv, d, L_max,
+        float(scale), _dtype(k_cache), _ptr(out), _ptr(status), _stream(stream)))
     return out
 
 

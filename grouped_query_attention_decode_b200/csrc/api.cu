@@ -232,6 +232,7 @@ extern "C" const char *gqa_status_string(int code) {
         case GQA_ERR_WORKSPACE: return "workspace is NULL or too small";
         case GQA_ERR_CUDA: return "a CUDA runtime call failed";
         case GQA_ERR_NO_DEVICE: return "no usable sm_100 device is current";
+        case GQA_ERR_SCRATCH_LIMIT: return "sizes need more scratch than the library's fixed no-allocation array";
         default: return "unknown status code";
     }
 }

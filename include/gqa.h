@@ -27,7 +27,8 @@
  *   - d is 64 or 128.  q, k_new, v_new and the caches share one element type (gqa_dtype_t).
  *   - Device pointers must be 16-byte aligned; `workspace` must be 256-byte aligned.
  *   - The caller owns and allocates every buffer, including the decode workspace.  The
- *     library allocates no device memory and keeps no per-call state.
+ *     library calls no device allocator and keeps no per-call state; its only device memory
+ *     is the fixed scratch array behind gqa_decode_noalloc.
  *   - Calls are asynchronous on `stream` (0 = the legacy default stream) and never
  *     synchronize the host.  Errors the host can see (a NULL pointer, a bad shape, a
  *     misaligned pointer, a short workspace) return a negative GQA_ERR_* code before anything
@@ -65,6 +66,8 @@ typedef enum {
 #define GQA_ERR_WORKSPACE (-7)            /* workspace NULL or smaller than required */
 #define GQA_ERR_CUDA (-8)                 /* a CUDA runtime call failed */
 #define GQA_ERR_NO_DEVICE (-9)            /* no usable sm_100 device is current */
+#define GQA_ERR_SCRATCH_LIMIT (-10)       /* gqa_decode_noalloc: the sizes need more scratch than
+                                             GQA_NOALLOC_SCRATCH_BYTES */
 
 /* Device-side status bits (OR-ed into *status). */
 #define GQA_STATUS_APPEND_OVERFLOW 1  /* gqa_kv_append: seq_lens[b] < 0 or >= L_max; row skipped */
@@ -127,6 +130,33 @@ int gqa_decode(const void *q, const void *k_cache, const void *v_cache, const in
                int B, int H_q, int H_kv, int d, int L_max, float scale, gqa_dtype_t dtype,
                float *out, void *workspace, size_t workspace_bytes, int32_t *status,
                cudaStream_t stream);
+
+/*
+ * gqa_decode_noalloc: gqa_decode without a caller-provided workspace.  (The pages have no
+ * counterpart of this call; it exists for callers, not for the method.)
+ *
+ * For callers that cannot allocate device memory for the workspace: a plugin inside a host
+ * framework that owns every device allocation, or a serving loop that must not call cudaMalloc
+ * (it can synchronize the device) and has no buffer of its own to lend.  The workspace is a
+ * fixed array of GQA_NOALLOC_SCRATCH_BYTES of device memory inside the library; every GPU that
+ * loads the library holds it until the process exits.  Arguments and results are those of
+ * gqa_decode; the caller still provides q, the caches, seq_lens and out.
+ *
+ *   - Sizes whose gqa_decode_workspace_size() exceeds GQA_NOALLOC_SCRATCH_BYTES are refused
+ *     with GQA_ERR_SCRATCH_LIMIT before anything runs (use gqa_decode with a workspace).
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
+ *     with that device current and caches it; make that first call before any stream capture.
+ *   - Nothing in the array needs to start at zero: each call writes what it later reads.
+ *   - Every call shares the one array and it keeps the last call's contents.  Two calls that
+ *     may overlap on the GPU (different streams, or different host threads without ordering)
+ *     race on it and produce wrong results; order them on one stream.
+ * No cudaMalloc, cudaFree or other allocating routine is called.
+ */
+#define GQA_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+int gqa_decode_noalloc(const void *q, const void *k_cache, const void *v_cache,
+                       const int32_t *seq_lens, int B, int H_q, int H_kv, int d, int L_max,
+                       float scale, gqa_dtype_t dtype, float *out, int32_t *status,
+                       cudaStream_t stream);
 
 /* gqa_status_string: a static, human-readable string for a GQA_OK / GQA_ERR_* code. */
 const char *gqa_status_string(int code);

@@ -36,7 +36,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_status_strings(lib):
-    for code in range(-9, 1):
+    for code in range(-10, 1):
         s = gqa.status_string(code)
         assert s and s != "unknown status code", code
     assert gqa.status_string(5) == "unknown status code"
