@@ -199,7 +199,7 @@ extern "C" int gqa_decode(const void *q, const void *k_cache, const void *v_cach
     const bool profile = ev0 != nullptr && ev1 != nullptr;
     int res;
     if (dtype == GQA_DTYPE_BF16) {
-        const int rp = g.RB <= 16 ? 16 : (g.RB <= 32 ? 32 : 64);
+        const int rp = tc_q_box_rows(g.RB);
         if (encode_fn() == nullptr) return GQA_ERR_CUDA;
         TmaMaps maps;
         if (!encode_q_map(&maps.q, q, B, H_q, d, rp) ||
@@ -209,7 +209,7 @@ extern "C" int gqa_decode(const void *q, const void *k_cache, const void *v_cach
             !encode_cache_map(&maps.v8, v_cache, B, H_kv, d, L_max, 8))
             return GQA_ERR_SHAPE;
         if (profile && cudaEventRecord(ev0, stream) != cudaSuccess) return GQA_ERR_CUDA;
-        res = launch_split_tc(maps, p, rp, stream);
+        res = launch_split_tc(maps, p, stream);
     } else {
         if (profile && cudaEventRecord(ev0, stream) != cudaSuccess) return GQA_ERR_CUDA;
         res = launch_split_f32(p, static_cast<const float *>(q), static_cast<const float *>(k_cache),

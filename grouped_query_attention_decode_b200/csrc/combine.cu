@@ -18,6 +18,8 @@
 namespace gqa {
 
 __global__ void __launch_bounds__(256) combine_kernel(const DecodeParams p) {
+    extern __shared__ int piece_cta[];  // CTA index of each piece of this unit, in line order
+    __shared__ int s_pieces;
     grid_dependency_wait();
     const int u = blockIdx.x;
     const int b = u / p.UB;
@@ -37,22 +39,36 @@ __global__ void __launch_bounds__(256) combine_kernel(const DecodeParams p) {
     }
     const long long total = hdr[p.B];
     const long long uoff = hdr[b] + static_cast<long long>(k) * nt;
-    const long long i0 = cta_of_tile(uoff, total, p.G);
-    const long long i1 = cta_of_tile(uoff + nt - 1, total, p.G);
-    if (i0 == i1) return;
-    const float *slots = p.ws + p.hdr_floats;
+    const int i0 = static_cast<int>(cta_of_tile(uoff, total, p.G));
+    const int i1 = static_cast<int>(cta_of_tile(uoff + nt - 1, total, p.G));
+    if (i0 == i1) return;  // one piece: the split kernel wrote the output
+    // Every CTA in [i0, i1] holds a piece of this unit unless its range is empty, which can only
+    // happen when there are fewer tiles than CTAs.
+    if (total >= p.G) {
+        for (int i = threadIdx.x; i <= i1 - i0; i += blockDim.x) piece_cta[i] = i0 + i;
+        if (threadIdx.x == 0) s_pieces = i1 - i0 + 1;
+    } else {
+        for (int i = threadIdx.x; i <= i1 - i0; i += blockDim.x)
+            piece_cta[i] = cta_range_begin(i0 + i, total, p.G) < cta_range_begin(i0 + i + 1, total, p.G) ? i0 + i : -1;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            int c = 0;
+            for (int i = 0; i <= i1 - i0; ++i)
+                if (piece_cta[i] >= 0) piece_cta[c++] = piece_cta[i];
+            s_pieces = c;
+        }
+    }
+    __syncthreads();
+    const int np = s_pieces;
+    const float *slots = p.ws + p.hdr_floats + static_cast<long long>(u) * p.slot_floats;
     for (int idx = threadIdx.x; idx < nh * d; idx += blockDim.x) {
         const int h = idx / d;
         float M = -INFINITY;
-        for (long long i = i0; i <= i1; ++i) {
-            if (cta_range_begin(i, total, p.G) == cta_range_begin(i + 1, total, p.G)) continue;
-            const float *s = slots + (i + u) * p.slot_floats;
-            M = fmaxf(M, s[nh * d + h]);
-        }
+        for (int j = 0; j < np; ++j)
+            M = fmaxf(M, slots[static_cast<long long>(piece_cta[j]) * p.slot_floats + nh * d + h]);
         float num = 0.f, den = 0.f;
-        for (long long i = i0; i <= i1; ++i) {
-            if (cta_range_begin(i, total, p.G) == cta_range_begin(i + 1, total, p.G)) continue;
-            const float *s = slots + (i + u) * p.slot_floats;
+        for (int j = 0; j < np; ++j) {
+            const float *s = slots + static_cast<long long>(piece_cta[j]) * p.slot_floats;
             const float wgt = ex2_approx(s[nh * d + h] - M);
             num = fmaf(wgt, s[idx], num);
             den = fmaf(wgt, s[nh * d + nh + h], den);
@@ -67,7 +83,7 @@ int launch_combine(const DecodeParams &p, cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(units));
     cfg.blockDim = dim3(256);
-    cfg.dynamicSmemBytes = 0;
+    cfg.dynamicSmemBytes = static_cast<size_t>(p.G) * sizeof(int);
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -8,15 +8,16 @@
 //
 //   S^T[128 rows x RP heads] = K_tile[128 x d] . Q^T            (UMMA, M=128, N=RP, K=d)
 //   softmax over the 128 rows, online across tiles, in fp32      (4 warps, one row per thread)
-//   O^T[d x RP] = V_tile^T[d x 128] . P^T[128 x RP]              (UMMA, M=d, N=RP, K=128)
+//   O^T[d x 2RP] = V_tile^T[d x 128] . [P_hi | P_lo]^T           (UMMA, M=d, N=2RP, K=128)
 //
 // and the O^T tiles are accumulated with the online-softmax rescale in registers (thread =
 // one of the d output columns).  P enters the second product as two bf16 parts (high, and the
-// rounding residual) that accumulate into the same TMEM tile, so it carries ~16 significant
-// bits rather than 8.  RP is the group's head count padded to 16/32/64; padded heads are
-// computed and ignored.  Roles (192 threads):
+// rounding residual) side by side, summed when the tile is read back, so it carries ~16
+// significant bits rather than 8.  NH is the group's head count rounded up to a power of two
+// (1..64) and RP = max(16, NH) the UMMA N; padded heads are computed and ignored.
+// Roles (192 threads):
 //   warp 0       TMA producer (q of each unit, K/V tiles); also owns the tensor memory
-//   warp 1       UMMA issuer (one elected thread)
+//   warp 1       UMMA issuer (one elected thread, event loop)
 //   warps 2..5   softmax / accumulation / epilogue (128 threads)
 // Every wait is bounded; on a timeout the CTA drains its in-flight copies and UMMAs, frees
 // its tensor memory, sets GQA_STATUS_WAIT_TIMEOUT and returns.
@@ -31,18 +32,25 @@ namespace gqa {
 
 constexpr unsigned long long kDrainNs = 1000000000ull;  // bound for draining in-flight work
 
-template <int D, int RP>
+template <int D, int NH>
 struct TcCfg {
+    static constexpr int RP = NH < 16 ? 16 : NH;      // UMMA N of S^T = K.Q^T
     static constexpr int T = 128;
     static constexpr int KB = D / 64;                 // 128-byte column blocks of a row
     static constexpr int TILE_BYTES = T * D * 2;      // one K or V tile
     static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
     static constexpr int Q_BYTES = RP * D * 2;
-    static constexpr int P_HALF = RP * T * 2;         // P^T in bf16: high part, then low part
-    static constexpr int P_BYTES = 2 * P_HALF;
-    static constexpr int TMEM_COLS = 4 * RP;          // S^T x2, O^T x2
+    // P^T in bf16 as 2*RP rows (heads' high parts, then their low parts) x T columns
+    static constexpr int P_BYTES = 2 * RP * T * 2;
+    // TMEM columns: S^T (RP) x2 buffers, then O^T (2*RP: high, low) x2 buffers
+    static constexpr int O_COL = 2 * RP;
+    static constexpr int TMEM_COLS = 6 * RP <= 128 ? 128 : (6 * RP <= 256 ? 256 : 512);
     static constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, RP, false, false);
-    static constexpr uint32_t IDESC_PV = idesc_bf16_f32(D, RP, true, false);
+    static constexpr uint32_t IDESC_PV = idesc_bf16_f32(D, 2 * RP, true, false);
+    // Running max and rescale factors live in registers up to 32 heads; with 64 heads they go
+    // through shared memory to keep the softmax threads under the register limit.
+    static constexpr bool REG_STATE = NH <= 32;
+    static constexpr int NH4 = (NH + 3) / 4;
 
     struct Small {
         uint64_t kv_full[8], kv_empty[8];
@@ -54,10 +62,10 @@ struct TcCfg {
         int b0;
         int pad_;
         long long begin, end, off0;
-        float wmax[2][4][RP];
-        float mcur[2][RP];
-        float alpha[2][RP];
-        float lsum[4][RP];
+        float4 wmax[2][4][NH4];  // per tile parity, warp: the warp's per-head maxima
+        float mcur[2][NH];       // 64-head path only
+        float alpha[2][NH];      // 64-head path only
+        float lsum[4][NH];
     };
 
     static constexpr int SMEM_LIMIT = 232448;
@@ -69,17 +77,24 @@ struct TcCfg {
     static constexpr int S = S_FIT > 6 ? 6 : S_FIT;
     static constexpr int SMEM_BYTES = S * STAGE_BYTES + FIXED;
     static_assert(S >= 2, "shared memory too small for a double-buffered ring");
-    static_assert(Q_BYTES % 1024 == 0 && P_HALF % 1024 == 0 && STAGE_BYTES % 1024 == 0, "");
+    static_assert(Q_BYTES % 1024 == 0 && P_BYTES % 1024 == 0 && STAGE_BYTES % 1024 == 0, "");
 };
 
-template <int D, int RP>
+// Add a byte offset to a shared-memory descriptor's start address (bits 0-13, 16-byte units).
+// Shared addresses stay below 2^18, so the field cannot carry into the next one.
+__device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t bytes) {
+    return desc + static_cast<uint64_t>(bytes >> 4);
+}
+
+template <int D, int NH>
 __global__ void __launch_bounds__(192, 1)
 split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_k8, const __grid_constant__ CUtensorMap tm_v,
                 const __grid_constant__ CUtensorMap tm_v8, const DecodeParams p) {
-    using C = TcCfg<D, RP>;
+    using C = TcCfg<D, NH>;
     constexpr int T = C::T;
     constexpr int S = C::S;
+    constexpr int RP = C::RP;
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t *const st_base = smem;
     uint8_t *const q_base = smem + S * C::STAGE_BYTES;
@@ -217,70 +232,88 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------------ UMMA issuer
+        // An event loop: a tile's S^T = K.Q^T is issued once its K/V stage has landed and its
+        // S buffer is free; its O^T = V^T.P^T once the softmax warps have written its P.  Each
+        // is issued as soon as it is ready, so releasing a stage never waits for the next
+        // tile's data to arrive.
         if (lane == 0) {
+            // K tile and Q: K-major (rows / heads by d), 8-row groups 1024 B apart.
+            // V^T: MN-major (d by rows): the two 64-column blocks T*128 B apart.
+            // P^T: K-major (2*RP rows by tile rows).
+            const uint64_t dk0 = sdesc_sw128(smem_u32(st_base), 16, 1024);
+            const uint64_t dv0 = sdesc_sw128(smem_u32(st_base + C::TILE_BYTES), T * 128, 1024);
+            const uint64_t dq0 = sdesc_sw128(smem_u32(q_base), 16, 1024);
+            const uint64_t dp0 = sdesc_sw128(smem_u32(p_base), 16, 1024);
             SegmentWalker w;
             w.init(p, cr);
             Segment sg;
-            int i = 0, sidx = 0, pv_next = 0;
+            bool qk_more = w.next(sg);
+            int qk_t = 0, qk_jj = 0, sidx = 0, pv_t = 0;
+            bool q_ready = false;
             bool ok = true;
-            auto issue_pv = [&](int t) -> bool {
-                const int j2 = t & 1;
-                if (!wait_bounded(&sm->p_full[j2], (t >> 1) & 1, abort_flag, budget)) return false;
-                if (t >= 2 && !wait_bounded(&sm->o_empty[j2], ((t >> 1) - 1) & 1, abort_flag, budget)) return false;
-                tc_fence_after_sync();
-                const uint32_t vaddr = smem_u32(st_base + (t % S) * C::STAGE_BYTES + C::TILE_BYTES);
-                const uint32_t paddr = smem_u32(p_base + j2 * C::P_BYTES);
-                // O^T = V^T . (P_hi + P_lo)^T: the two bf16 parts of P accumulate into one tile,
-                // so P enters the product with ~16 significant bits instead of 8.
+            uint64_t idle_since = global_timer_ns();
+            uint32_t idle_polls = 0;
+            while (qk_more || pv_t < qk_t) {
+                bool progress = false;
+                if (qk_more) {
+                    const int qb = sidx % C::QB;
+                    if (!q_ready) q_ready = mbar_test_wait(&sm->q_full[qb], (sidx / C::QB) & 1);
+                    const int st = qk_t % S;
+                    const int j2 = qk_t & 1;
+                    if (q_ready && mbar_test_wait(&sm->kv_full[st], (qk_t / S) & 1) &&
+                        (qk_t < 2 || mbar_test_wait(&sm->s_empty[j2], ((qk_t >> 1) - 1) & 1))) {
+                        tc_fence_after_sync();
+                        const uint64_t dk = desc_add(dk0, st * C::STAGE_BYTES);
+                        const uint64_t dq = desc_add(dq0, qb * C::Q_BYTES);
 #pragma unroll
-                for (int part = 0; part < 2; ++part) {
-#pragma unroll
-                    for (int kk = 0; kk < T / 16; ++kk) {
-                        // V^T: M = d (contiguous within 128-byte rows), K = rows; MN-major.
-                        const uint64_t a = sdesc_sw128(vaddr + kk * 2048, T * 128, 1024);
-                        // P^T: N = heads, K = rows; K-major, 64 rows per 128-byte swizzle row.
-                        const uint64_t bdesc = sdesc_sw128(paddr + part * C::P_HALF + (kk >> 2) * RP * 128 + (kk & 3) * 32, 16, 1024);
-                        umma_bf16(tmem + 2 * RP + j2 * RP, a, bdesc, C::IDESC_PV, (part | kk) ? 1u : 0u);
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t off_k = (kk >> 2) * T * 128 + (kk & 3) * 32;
+                            const uint32_t off_q = (kk >> 2) * RP * 128 + (kk & 3) * 32;
+                            umma_bf16(tmem + j2 * RP, desc_add(dk, off_k), desc_add(dq, off_q),
+                                      C::IDESC_QK, kk > 0 ? 1u : 0u);
+                        }
+                        umma_commit(&sm->s_full[j2]);
+                        ++qk_t;
+                        if (++qk_jj == sg.len) {
+                            umma_commit(&sm->q_empty[qb]);
+                            ++sidx;
+                            qk_jj = 0;
+                            q_ready = false;
+                            qk_more = w.next(sg);
+                        }
+                        progress = true;
                     }
                 }
-                umma_commit(&sm->o_full[j2]);
-                umma_commit(&sm->kv_empty[t % S]);
-                return true;
-            };
-            while (ok && w.next(sg)) {
-                const int qb = sidx % C::QB;
-                if (!wait_bounded(&sm->q_full[qb], (sidx / C::QB) & 1, abort_flag, budget)) {
-                    ok = false;
-                    break;
-                }
-                const uint32_t qaddr = smem_u32(q_base + qb * C::Q_BYTES);
-                for (int jj = 0; jj < sg.len; ++jj, ++i) {
-                    const int st = i % S;
-                    const int j2 = i & 1;
-                    if (!wait_bounded(&sm->kv_full[st], (i / S) & 1, abort_flag, budget)) { ok = false; break; }
-                    if (i >= 2 && !wait_bounded(&sm->s_empty[j2], ((i >> 1) - 1) & 1, abort_flag, budget)) { ok = false; break; }
-                    tc_fence_after_sync();
-                    const uint32_t kaddr = smem_u32(st_base + st * C::STAGE_BYTES);
+                if (pv_t < qk_t) {
+                    const int j2 = pv_t & 1;
+                    if (mbar_test_wait(&sm->p_full[j2], (pv_t >> 1) & 1) &&
+                        (pv_t < 2 || mbar_test_wait(&sm->o_empty[j2], ((pv_t >> 1) - 1) & 1))) {
+                        tc_fence_after_sync();
+                        const uint64_t dv = desc_add(dv0, (pv_t % S) * C::STAGE_BYTES);
+                        const uint64_t dp = desc_add(dp0, j2 * C::P_BYTES);
+                        // O^T[:, 0:RP] = V^T.P_hi^T and O^T[:, RP:2RP] = V^T.P_lo^T in one
+                        // N = 2*RP product.
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        // K tile: M = rows, K = d; K-major.  Q: N = heads, K = d; K-major.
-                        const uint64_t a = sdesc_sw128(kaddr + (kk >> 2) * T * 128 + (kk & 3) * 32, 16, 1024);
-                        const uint64_t bdesc = sdesc_sw128(qaddr + (kk >> 2) * RP * 128 + (kk & 3) * 32, 16, 1024);
-                        umma_bf16(tmem + j2 * RP, a, bdesc, C::IDESC_QK, kk > 0 ? 1u : 0u);
-                    }
-                    umma_commit(&sm->s_full[j2]);
-                    const bool last = (jj == sg.len - 1);
-                    if (last) umma_commit(&sm->q_empty[qb]);
-                    if (pv_next < i) {
-                        if (!issue_pv(pv_next)) { ok = false; break; }
-                        ++pv_next;
-                    }
-                    if (last) {
-                        if (!issue_pv(i)) { ok = false; break; }
-                        pv_next = i + 1;
+                        for (int kk = 0; kk < T / 16; ++kk) {
+                            const uint32_t off_p = (kk >> 2) * 2 * RP * 128 + (kk & 3) * 32;
+                            umma_bf16(tmem + C::O_COL + j2 * C::O_COL, desc_add(dv, kk * 2048),
+                                      desc_add(dp, off_p), C::IDESC_PV, kk > 0 ? 1u : 0u);
+                        }
+                        umma_commit(&sm->o_full[j2]);
+                        umma_commit(&sm->kv_empty[pv_t % S]);
+                        ++pv_t;
+                        progress = true;
                     }
                 }
-                ++sidx;
+                if (progress) {
+                    idle_polls = 0;
+                } else if ((++idle_polls & 15u) == 0) {
+                    if (idle_polls == 16) idle_since = global_timer_ns();
+                    if (*abort_flag || global_timer_ns() - idle_since > budget) {
+                        ok = false;
+                        break;
+                    }
+                }
             }
             if (!ok) fail();
             umma_commit(&sm->mma_done);
@@ -294,19 +327,29 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const uint32_t lane_addr = static_cast<uint32_t>(q4 * 32) << 16;
         // Output column (of d) this thread accumulates: O^T row in TMEM.
         const int dcol = (D == 128) ? row : (lane < 16 ? q4 * 16 + lane : -1);
+        // Where this thread's row lands in P^T: column `row` of every head row.
+        const int col = row & 63;
+        const int chunk = col >> 3;
+        const int within = (col & 7) * 2;
         SegmentWalker w;
         w.init(p, cr);
         Segment sg;
         int i = 0;
         bool ok = true;
-        float O[RP];
-        float l[RP];
+        float O[NH];
+        float l[NH];
+        float m_run[C::REG_STATE ? NH : 1];
+        float alpha[C::REG_STATE ? NH : 1];
         while (ok && w.next(sg)) {
             const int nh = min(p.RB, p.r - sg.hb * p.RB);
 #pragma unroll
-            for (int h = 0; h < RP; ++h) {
+            for (int h = 0; h < NH; ++h) {
                 O[h] = 0.f;
                 l[h] = 0.f;
+            }
+            if constexpr (C::REG_STATE) {
+#pragma unroll
+                for (int h = 0; h < NH; ++h) m_run[h] = -INFINITY;
             }
             int j2 = 0;
             for (int jj = 0; jj < sg.len; ++jj, ++i) {
@@ -335,46 +378,84 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 if (lane == 0) mbar_arrive(&sm->s_empty[j2]);
 
                 const bool valid = row < rows;
-                float x[RP];
+                float x[NH];
 #pragma unroll
-                for (int h = 0; h < RP; ++h)
+                for (int h = 0; h < NH; ++h)
                     x[h] = valid ? __uint_as_float(sr[h]) * p.scale_log2 : -INFINITY;
+                // Per-head maximum over the warp's 32 rows: interleaved butterflies.
+                float wm[NH];
 #pragma unroll
-                for (int h = 0; h < RP; ++h) {
-                    if (h < nh) {
-                        const float wm = warp_max_f32(x[h]);
-                        if (lane == 0) sm->wmax[j2][q4][h] = wm;
-                    }
+                for (int h = 0; h < NH; ++h) wm[h] = x[h];
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) {
+#pragma unroll
+                    for (int h = 0; h < NH; ++h) wm[h] = fmaxf(wm[h], __shfl_xor_sync(kFullMask, wm[h], off));
                 }
-                named_bar_sync(1, 128);
-                if (wg_tid < nh) {
-                    const int h = wg_tid;
-                    const float tmax = fmaxf(fmaxf(sm->wmax[j2][0][h], sm->wmax[j2][1][h]),
-                                             fmaxf(sm->wmax[j2][2][h], sm->wmax[j2][3][h]));
-                    const float m_old = jj == 0 ? -INFINITY : sm->mcur[j2 ^ 1][h];
-                    const float m_new = fmaxf(m_old, tmax);
-                    sm->mcur[j2][h] = m_new;
-                    sm->alpha[j2][h] = jj == 0 ? 0.f : ex2_approx(m_old - m_new);
+                if (lane == 0) {
+                    float *dst = reinterpret_cast<float *>(&sm->wmax[j2][q4][0]);
+#pragma unroll
+                    for (int h = 0; h < NH; ++h) dst[h] = wm[h];
                 }
                 named_bar_sync(1, 128);
 
-                // P^T as bf16 high and low parts (P = hi + lo to ~16 bits), K-major with
-                // 128-byte swizzle: head h is row h, tile row r is column r (64 columns per
-                // 128-byte row, two column blocks).
-                uint8_t *pb = p_base + j2 * C::P_BYTES + (row >> 6) * RP * 128;
-                const int col = row & 63;
-                const int chunk = col >> 3;
-                const int within = (col & 7) * 2;
+                if constexpr (C::REG_STATE) {
+                    // Every thread forms the tile maximum of every head from the four warp
+                    // maxima and keeps the running maximum in registers (identical in all
+                    // threads), so one barrier per tile suffices.
 #pragma unroll
-                for (int h = 0; h < RP; ++h) {
+                    for (int h4 = 0; h4 < C::NH4; ++h4) {
+                        const float4 a = sm->wmax[j2][0][h4], b = sm->wmax[j2][1][h4];
+                        const float4 c = sm->wmax[j2][2][h4], e = sm->wmax[j2][3][h4];
+                        const float t4[4] = {fmaxf(fmaxf(a.x, b.x), fmaxf(c.x, e.x)),
+                                             fmaxf(fmaxf(a.y, b.y), fmaxf(c.y, e.y)),
+                                             fmaxf(fmaxf(a.z, b.z), fmaxf(c.z, e.z)),
+                                             fmaxf(fmaxf(a.w, b.w), fmaxf(c.w, e.w))};
+#pragma unroll
+                        for (int e4 = 0; e4 < 4; ++e4) {
+                            const int h = h4 * 4 + e4;
+                            if (h < NH) {
+                                const float m_new = fmaxf(m_run[h], t4[e4]);
+                                alpha[h] = m_new == -INFINITY ? 0.f : ex2_approx(m_run[h] - m_new);
+                                m_run[h] = m_new;
+                            }
+                        }
+                    }
+                } else {
+                    if (wg_tid < nh) {
+                        const int h = wg_tid;
+                        const float *wf = reinterpret_cast<const float *>(&sm->wmax[j2][0][0]);
+                        constexpr int WS = 4 * C::NH4;  // floats per warp row
+                        const float tmax = fmaxf(fmaxf(wf[h], wf[WS + h]), fmaxf(wf[2 * WS + h], wf[3 * WS + h]));
+                        const float m_old = jj == 0 ? -INFINITY : sm->mcur[j2 ^ 1][h];
+                        const float m_new = fmaxf(m_old, tmax);
+                        sm->mcur[j2][h] = m_new;
+                        sm->alpha[j2][h] = jj == 0 ? 0.f : ex2_approx(m_old - m_new);
+                    }
+                    named_bar_sync(1, 128);
+                }
+
+                // P^T as bf16 high and low parts (P = hi + lo to ~16 bits), K-major with
+                // 128-byte swizzle: row h holds head h's high parts, row RP + h its low parts,
+                // tile row r is column r (64 columns per 128-byte row, two column blocks).
+                uint8_t *pb = p_base + j2 * C::P_BYTES + (row >> 6) * 2 * RP * 128;
+#pragma unroll
+                for (int h = 0; h < NH; ++h) {
+                    float m_h, a_h;
+                    if constexpr (C::REG_STATE) {
+                        m_h = m_run[h];
+                        a_h = alpha[h];
+                    } else {
+                        m_h = sm->mcur[j2][h];
+                        a_h = sm->alpha[j2][h];
+                    }
+                    const float pr = ex2_approx(x[h] - m_h);
+                    const __nv_bfloat16 hi = __float2bfloat16_rn(pr);
+                    const __nv_bfloat16 lo = __float2bfloat16_rn(pr - __bfloat162float(hi));
+                    l[h] = l[h] * a_h + pr;
                     if (h < nh) {
-                        const float pr = ex2_approx(x[h] - sm->mcur[j2][h]);
-                        const __nv_bfloat16 hi = __float2bfloat16_rn(pr);
-                        const __nv_bfloat16 lo = __float2bfloat16_rn(pr - __bfloat162float(hi));
-                        l[h] = l[h] * sm->alpha[j2][h] + pr;
                         uint8_t *dst = pb + h * 128 + ((chunk ^ (h & 7)) << 4) + within;
                         *reinterpret_cast<__nv_bfloat16 *>(dst) = hi;
-                        *reinterpret_cast<__nv_bfloat16 *>(dst + C::P_HALF) = lo;
+                        *reinterpret_cast<__nv_bfloat16 *>(dst + RP * 128) = lo;
                     }
                 }
                 fence_proxy_async_smem();
@@ -387,15 +468,26 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     const int t = i - 1, jt = t & 1;
                     if (!wait_bounded(&sm->o_full[jt], (t >> 1) & 1, abort_flag, budget)) { ok = false; break; }
                     tc_fence_after_sync();
-                    uint32_t orr[RP];
-                    tmem_ld_cols<RP>(tmem + lane_addr + 2 * RP + jt * RP, orr);
-                    tmem_wait_ld();
+                    const uint32_t obase = tmem + lane_addr + C::O_COL + jt * C::O_COL;
+#pragma unroll
+                    for (int c = 0; c < NH; c += 16) {
+                        uint32_t hi[16], lo[16];
+                        tmem_ld16(obase + c, hi);
+                        tmem_ld16(obase + RP + c, lo);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            if (c + e < NH) {
+                                float a_h;
+                                if constexpr (C::REG_STATE) a_h = alpha[c + e];
+                                else a_h = sm->alpha[j2][c + e];
+                                O[c + e] = (O[c + e] + (__uint_as_float(hi[e]) + __uint_as_float(lo[e]))) * a_h;
+                            }
+                        }
+                    }
                     tc_fence_before_sync();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&sm->o_empty[jt]);
-#pragma unroll
-                    for (int h = 0; h < RP; ++h)
-                        if (h < nh) O[h] = (O[h] + __uint_as_float(orr[h])) * sm->alpha[j2][h];
                 }
             }
             if (!ok) break;
@@ -404,23 +496,26 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const int t = i - 1, jt = t & 1;
                 if (!wait_bounded(&sm->o_full[jt], (t >> 1) & 1, abort_flag, budget)) { ok = false; break; }
                 tc_fence_after_sync();
-                uint32_t orr[RP];
-                tmem_ld_cols<RP>(tmem + lane_addr + 2 * RP + jt * RP, orr);
-                tmem_wait_ld();
+                const uint32_t obase = tmem + lane_addr + C::O_COL + jt * C::O_COL;
+#pragma unroll
+                for (int c = 0; c < NH; c += 16) {
+                    uint32_t hi[16], lo[16];
+                    tmem_ld16(obase + c, hi);
+                    tmem_ld16(obase + RP + c, lo);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        if (c + e < NH) O[c + e] += __uint_as_float(hi[e]) + __uint_as_float(lo[e]);
+                }
                 tc_fence_before_sync();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm->o_empty[jt]);
-#pragma unroll
-                for (int h = 0; h < RP; ++h)
-                    if (h < nh) O[h] += __uint_as_float(orr[h]);
             }
             // Sum of the softmax numerators over the 128 rows of every tile of the piece.
 #pragma unroll
-            for (int h = 0; h < RP; ++h) {
-                if (h < nh) {
-                    const float s = warp_sum_f32(l[h]);
-                    if (lane == 0) sm->lsum[q4][h] = s;
-                }
+            for (int h = 0; h < NH; ++h) {
+                const float s = warp_sum_f32(l[h]);
+                if (lane == 0 && h < nh) sm->lsum[q4][h] = s;
             }
             named_bar_sync(1, 128);
             if (dcol >= 0) {
@@ -428,7 +523,7 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 if (sg.whole) {
                     float *o = p.out + (static_cast<long long>(sg.b) * p.H_q + h0) * D + dcol;
 #pragma unroll
-                    for (int h = 0; h < RP; ++h) {
+                    for (int h = 0; h < NH; ++h) {
                         if (h < nh) {
                             const float L = sm->lsum[0][h] + sm->lsum[1][h] + sm->lsum[2][h] + sm->lsum[3][h];
                             o[static_cast<long long>(h) * D] = O[h] / L;
@@ -438,15 +533,25 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     float *slot = p.ws + p.hdr_floats +
                                   (static_cast<long long>(blockIdx.x) + sg.unit) * p.slot_floats;
 #pragma unroll
-                    for (int h = 0; h < RP; ++h)
+                    for (int h = 0; h < NH; ++h)
                         if (h < nh) slot[h * D + dcol] = O[h];
                     if (dcol < nh) {
                         const int h = dcol;
-                        slot[nh * D + h] = sm->mcur[j2][h];
+                        float m_final = -INFINITY;
+                        if constexpr (C::REG_STATE) {
+#pragma unroll
+                            for (int hh = 0; hh < NH; ++hh)
+                                if (hh == h) m_final = m_run[hh];
+                        } else {
+                            m_final = sm->mcur[j2][h];
+                        }
+                        slot[nh * D + h] = m_final;
                         slot[nh * D + nh + h] = sm->lsum[0][h] + sm->lsum[1][h] + sm->lsum[2][h] + sm->lsum[3][h];
                     }
                 }
             }
+            // the next piece rewrites lsum only after every thread has read it
+            named_bar_sync(1, 128);
         }
         if (!ok) fail();
     }
@@ -457,10 +562,10 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (warp == 0) tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
-template <int D, int RP>
+template <int D, int NH>
 static int launch_split_tc_impl(const TmaMaps &maps, const DecodeParams &p, cudaStream_t stream) {
-    using C = TcCfg<D, RP>;
-    auto kern = split_tc_kernel<D, RP>;
+    using C = TcCfg<D, NH>;
+    auto kern = split_tc_kernel<D, NH>;
     static bool attr_set[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return GQA_ERR_CUDA;
@@ -484,15 +589,36 @@ static int launch_split_tc_impl(const TmaMaps &maps, const DecodeParams &p, cuda
     return GQA_OK;
 }
 
-int launch_split_tc(const TmaMaps &maps, const DecodeParams &p, int rp, cudaStream_t stream) {
-    if (p.d == 128) {
-        if (rp == 16) return launch_split_tc_impl<128, 16>(maps, p, stream);
-        if (rp == 32) return launch_split_tc_impl<128, 32>(maps, p, stream);
-        return launch_split_tc_impl<128, 64>(maps, p, stream);
+template <int D>
+static int launch_split_tc_d(const TmaMaps &maps, const DecodeParams &p, int nh, cudaStream_t stream) {
+    switch (nh) {
+        case 1: return launch_split_tc_impl<D, 1>(maps, p, stream);
+        case 2: return launch_split_tc_impl<D, 2>(maps, p, stream);
+        case 4: return launch_split_tc_impl<D, 4>(maps, p, stream);
+        case 8: return launch_split_tc_impl<D, 8>(maps, p, stream);
+        case 16: return launch_split_tc_impl<D, 16>(maps, p, stream);
+        case 32: return launch_split_tc_impl<D, 32>(maps, p, stream);
+        default: return launch_split_tc_impl<D, 64>(maps, p, stream);
     }
-    if (rp == 16) return launch_split_tc_impl<64, 16>(maps, p, stream);
-    if (rp == 32) return launch_split_tc_impl<64, 32>(maps, p, stream);
-    return launch_split_tc_impl<64, 64>(maps, p, stream);
+}
+
+// Query heads per unit rounded up to a power of two (the kernel's compile-time head count).
+int tc_heads_bucket(int heads_per_unit) {
+    int nh = 1;
+    while (nh < heads_per_unit) nh <<= 1;
+    return nh;
+}
+
+// Rows of the q TMA box: the UMMA N of S^T = K.Q^T.
+int tc_q_box_rows(int heads_per_unit) {
+    const int nh = tc_heads_bucket(heads_per_unit);
+    return nh < 16 ? 16 : nh;
+}
+
+int launch_split_tc(const TmaMaps &maps, const DecodeParams &p, cudaStream_t stream) {
+    const int nh = tc_heads_bucket(p.RB);
+    return p.d == 128 ? launch_split_tc_d<128>(maps, p, nh, stream)
+                      : launch_split_tc_d<64>(maps, p, nh, stream);
 }
 
 }  // namespace gqa

@@ -16,7 +16,8 @@ struct TmaMaps {
     CUtensorMap q, k, k8, v, v8;
 };
 
-int launch_split_tc(const TmaMaps &maps, const DecodeParams &p, int rp, cudaStream_t stream);
+int launch_split_tc(const TmaMaps &maps, const DecodeParams &p, cudaStream_t stream);
+int tc_q_box_rows(int heads_per_unit);
 int launch_split_f32(const DecodeParams &p, const float *q, const float *kc, const float *vc,
                      cudaStream_t stream);
 int launch_combine(const DecodeParams &p, cudaStream_t stream);
