@@ -352,13 +352,15 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 for (int h = 0; h < NH; ++h) m_run[h] = -INFINITY;
             }
             int j2 = 0;
+            // A failed wait sets `bad`; the threads then agree at the next named barrier
+            // (named_bar_any) and leave together, so no warp is left waiting at a barrier.
+            bool bad = false;
             for (int jj = 0; jj < sg.len; ++jj, ++i) {
                 j2 = i & 1;
                 const int rows = min(T, sg.n - (sg.j0 + jj) * T);
-                if (rows < T) {
+                if (rows < T && !bad && wait_bounded(&sm->kv_full[i % S], (i / S) & 1, abort_flag, budget)) {
                     // Rows past n: zero V in shared memory so that 0-weight rows add exactly 0
                     // (stale or unread data there may hold NaN or Inf).
-                    if (!wait_bounded(&sm->kv_full[i % S], (i / S) & 1, abort_flag, budget)) { ok = false; break; }
                     uint8_t *vbase = st_base + (i % S) * C::STAGE_BYTES + C::TILE_BYTES;
                     const int nchunks = (T - rows) * 8;  // 16-byte chunks per column block
                     for (int c = wg_tid; c < nchunks * C::KB; c += 128) {
@@ -367,15 +369,22 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         const int rr = rows + (rem >> 3);
                         *reinterpret_cast<uint4 *>(vbase + kb * T * 128 + rr * 128 + (rem & 7) * 16) = make_uint4(0, 0, 0, 0);
                     }
+                } else if (rows < T) {
+                    bad = true;
                 }
-                if (!wait_bounded(&sm->s_full[j2], (i >> 1) & 1, abort_flag, budget)) { ok = false; break; }
-                tc_fence_after_sync();
                 uint32_t sr[RP];
-                tmem_ld_cols<RP>(tmem + lane_addr + j2 * RP, sr);
-                tmem_wait_ld();
-                tc_fence_before_sync();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sm->s_empty[j2]);
+                if (!bad && wait_bounded(&sm->s_full[j2], (i >> 1) & 1, abort_flag, budget)) {
+                    tc_fence_after_sync();
+                    tmem_ld_cols<RP>(tmem + lane_addr + j2 * RP, sr);
+                    tmem_wait_ld();
+                    tc_fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sm->s_empty[j2]);
+                } else {
+                    bad = true;
+#pragma unroll
+                    for (int h = 0; h < RP; ++h) sr[h] = 0u;
+                }
 
                 const bool valid = row < rows;
                 float x[NH];
@@ -396,7 +405,10 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                     for (int h = 0; h < NH; ++h) dst[h] = wm[h];
                 }
-                named_bar_sync(1, 128);
+                if (named_bar_any(1, 128, bad)) {
+                    ok = false;
+                    break;
+                }
 
                 if constexpr (C::REG_STATE) {
                     // Every thread forms the tile maximum of every head from the four warp
@@ -431,7 +443,7 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         sm->mcur[j2][h] = m_new;
                         sm->alpha[j2][h] = jj == 0 ? 0.f : ex2_approx(m_old - m_new);
                     }
-                    named_bar_sync(1, 128);
+                    named_bar_sync(1, 128);  // every thread of the group arrives here
                 }
 
                 // P^T as bf16 high and low parts (P = hi + lo to ~16 bits), K-major with
@@ -466,7 +478,10 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     // O(i-1) was computed against the previous max; fold it in and move the
                     // running sum to the current max.
                     const int t = i - 1, jt = t & 1;
-                    if (!wait_bounded(&sm->o_full[jt], (t >> 1) & 1, abort_flag, budget)) { ok = false; break; }
+                    if (!wait_bounded(&sm->o_full[jt], (t >> 1) & 1, abort_flag, budget)) {
+                        bad = true;
+                        continue;
+                    }
                     tc_fence_after_sync();
                     const uint32_t obase = tmem + lane_addr + C::O_COL + jt * C::O_COL;
 #pragma unroll
@@ -491,10 +506,9 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
             }
             if (!ok) break;
-            {
+            if (!bad && wait_bounded(&sm->o_full[(i - 1) & 1], ((i - 1) >> 1) & 1, abort_flag, budget)) {
                 // Last tile of the piece: its O is already relative to the final max.
-                const int t = i - 1, jt = t & 1;
-                if (!wait_bounded(&sm->o_full[jt], (t >> 1) & 1, abort_flag, budget)) { ok = false; break; }
+                const int jt = (i - 1) & 1;
                 tc_fence_after_sync();
                 const uint32_t obase = tmem + lane_addr + C::O_COL + jt * C::O_COL;
 #pragma unroll
@@ -510,6 +524,8 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tc_fence_before_sync();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm->o_empty[jt]);
+            } else {
+                bad = true;
             }
             // Sum of the softmax numerators over the 128 rows of every tile of the piece.
 #pragma unroll
@@ -517,7 +533,10 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const float s = warp_sum_f32(l[h]);
                 if (lane == 0 && h < nh) sm->lsum[q4][h] = s;
             }
-            named_bar_sync(1, 128);
+            if (named_bar_any(1, 128, bad)) {
+                ok = false;
+                break;
+            }
             if (dcol >= 0) {
                 const int h0 = sg.kvh * p.r + sg.hb * p.RB;
                 if (sg.whole) {
