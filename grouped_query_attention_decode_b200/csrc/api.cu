@@ -189,7 +189,10 @@ extern "C" int gqa_decode(const void *q, const void *k_cache, const void *v_cach
     p.HB = g.HB;
     p.UB = g.UB;
     p.T = dtype == GQA_DTYPE_BF16 ? 128 : 64;
-    p.G = sms;
+    // One persistent CTA per SM, but never more CTAs than the largest possible tile count
+    // (the workspace is sized for one per SM, which bounds this).
+    const long long max_tiles = g.units * ((static_cast<long long>(L_max) + p.T - 1) / p.T);
+    p.G = max_tiles < sms ? static_cast<int>(max_tiles) : sms;
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     p.wait_ns = g_wait_ns.load();
     p.slot_floats = g.slot_floats;

@@ -17,8 +17,15 @@
 
 namespace gqa {
 
-__global__ void __launch_bounds__(256) combine_kernel(const DecodeParams p) {
-    extern __shared__ int piece_cta[];  // CTA index of each piece of this unit, in line order
+constexpr int kCombineThreads = 256;
+constexpr int kCombineOutputsPerCta = 4 * kCombineThreads;
+
+// grid = (units, chunks of kCombineOutputsPerCta outputs of one unit)
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(const DecodeParams p) {
+    extern __shared__ float csm[];
+    int *piece_cta = reinterpret_cast<int *>(csm);  // CTA index of each piece, in line order
+    float *wts = csm + p.G;                         // [piece][head] merge weight
+    float *mref = wts + static_cast<long long>(p.G) * p.RB;  // [piece][head] reference max
     __shared__ int s_pieces;
     grid_dependency_wait();
     const int u = blockIdx.x;
@@ -29,12 +36,15 @@ __global__ void __launch_bounds__(256) combine_kernel(const DecodeParams p) {
     const int nh = min(p.RB, p.r - hb * p.RB);
     const int h0 = kvh * p.r + hb * p.RB;
     const int d = p.d;
+    const int first = blockIdx.y * kCombineOutputsPerCta;
+    const int last = min(nh * d, first + kCombineOutputsPerCta);
+    if (first >= last) return;
     float *o = p.out + (static_cast<long long>(b) * p.H_q + h0) * d;
     const long long *hdr = reinterpret_cast<const long long *>(p.ws);
     const int n = valid_len(p.seq_lens[b], p.L_max);
     const int nt = tiles_of(n, p.T);
     if (nt == 0) {
-        for (int idx = threadIdx.x; idx < nh * d; idx += blockDim.x) o[idx] = 0.f;
+        for (int idx = first + threadIdx.x; idx < last; idx += blockDim.x) o[idx] = 0.f;
         return;
     }
     const long long total = hdr[p.B];
@@ -61,29 +71,51 @@ __global__ void __launch_bounds__(256) combine_kernel(const DecodeParams p) {
     __syncthreads();
     const int np = s_pieces;
     const float *slots = p.ws + p.hdr_floats + static_cast<long long>(u) * p.slot_floats;
-    for (int idx = threadIdx.x; idx < nh * d; idx += blockDim.x) {
-        const int h = idx / d;
+    // weights: w[c][h] = 2^(m_c - M) / sum_c' 2^(m_c' - M) l_c'
+    for (int idx = threadIdx.x; idx < np * nh; idx += blockDim.x) {
+        const int c = idx / nh, h = idx - c * nh;
+        const float *sl = slots + static_cast<long long>(piece_cta[c]) * p.slot_floats;
+        mref[idx] = sl[nh * d + h];
+        wts[idx] = sl[nh * d + nh + h];  // l_c for now
+    }
+    __syncthreads();
+    for (int h = threadIdx.x; h < nh; h += blockDim.x) {
         float M = -INFINITY;
-        for (int j = 0; j < np; ++j)
-            M = fmaxf(M, slots[static_cast<long long>(piece_cta[j]) * p.slot_floats + nh * d + h]);
-        float num = 0.f, den = 0.f;
-        for (int j = 0; j < np; ++j) {
-            const float *s = slots + static_cast<long long>(piece_cta[j]) * p.slot_floats;
-            const float wgt = ex2_approx(s[nh * d + h] - M);
-            num = fmaf(wgt, s[idx], num);
-            den = fmaf(wgt, s[nh * d + nh + h], den);
-        }
-        o[idx] = num / den;
+        for (int c = 0; c < np; ++c) M = fmaxf(M, mref[c * nh + h]);
+        float den = 0.f;
+        for (int c = 0; c < np; ++c) den = fmaf(ex2_approx(mref[c * nh + h] - M), wts[c * nh + h], den);
+        const float inv = 1.f / den;
+        for (int c = 0; c < np; ++c) wts[c * nh + h] = ex2_approx(mref[c * nh + h] - M) * inv;
+    }
+    __syncthreads();
+    for (int idx = first + threadIdx.x; idx < last; idx += blockDim.x) {
+        const int h = idx / d;
+        float acc = 0.f;
+#pragma unroll 4
+        for (int c = 0; c < np; ++c)
+            acc = fmaf(wts[c * nh + h], slots[static_cast<long long>(piece_cta[c]) * p.slot_floats + idx], acc);
+        o[idx] = acc;
     }
 }
 
 int launch_combine(const DecodeParams &p, cudaStream_t stream) {
     const long long units = static_cast<long long>(p.B) * p.UB;
     if (units == 0) return GQA_OK;
+    const int chunks = (p.RB * p.d + kCombineOutputsPerCta - 1) / kCombineOutputsPerCta;
+    const size_t smem = static_cast<size_t>(p.G) * (sizeof(int) + 2 * sizeof(float) * p.RB);
+    static size_t smem_set[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GQA_ERR_CUDA;
+    if (smem > 48 * 1024 && (dev >= 64 || smem_set[dev] < smem)) {
+        if (cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smem)) != cudaSuccess)
+            return GQA_ERR_CUDA;
+        if (dev < 64) smem_set[dev] = smem;
+    }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(units));
-    cfg.blockDim = dim3(256);
-    cfg.dynamicSmemBytes = static_cast<size_t>(p.G) * sizeof(int);
+    cfg.gridDim = dim3(static_cast<unsigned>(units), chunks);
+    cfg.blockDim = dim3(kCombineThreads);
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
