@@ -40,17 +40,23 @@ struct TcCfg {
     static constexpr int TILE_BYTES = T * D * 2;      // one K or V tile
     static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
     static constexpr int Q_BYTES = RP * D * 2;
-    // P^T in bf16 as 2*RP rows (heads' high parts, then their low parts) x T columns
+    // P^T in bf16, MN-major: tile row r (the K index) holds 2*RP values, the high parts of
+    // heads 0..RP-1 then their low parts.  Rows are 64 bytes (RP = 16, 64-byte swizzle) or
+    // 128 bytes (RP >= 32, 128-byte swizzle); 2*RP > 64 values take two 128-byte atoms.
+    static constexpr int P_ROWB = 4 * RP >= 128 ? 128 : 4 * RP;
+    static constexpr int P_ATOMB = T * P_ROWB;
+    static constexpr uint32_t P_LAYOUT = P_ROWB == 128 ? 2u : 4u;
     static constexpr int P_BYTES = 2 * RP * T * 2;
     // TMEM columns: S^T (RP) x2 buffers, then O^T (2*RP: high, low) x2 buffers
     static constexpr int O_COL = 2 * RP;
     static constexpr int TMEM_COLS = 6 * RP <= 128 ? 128 : (6 * RP <= 256 ? 256 : 512);
     static constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, RP, false, false);
-    static constexpr uint32_t IDESC_PV = idesc_bf16_f32(D, 2 * RP, true, false);
+    static constexpr uint32_t IDESC_PV = idesc_bf16_f32(D, 2 * RP, true, true);
     // Running max and rescale factors live in registers up to 32 heads; with 64 heads they go
     // through shared memory to keep the softmax threads under the register limit.
     static constexpr bool REG_STATE = NH <= 32;
     static constexpr int NH4 = (NH + 3) / 4;
+    static constexpr int LOG2NH = NH >= 64 ? 6 : NH >= 32 ? 5 : NH >= 16 ? 4 : NH >= 8 ? 3 : NH >= 4 ? 2 : NH >= 2 ? 1 : 0;
 
     struct Small {
         uint64_t kv_full[8], kv_empty[8];
@@ -79,6 +85,36 @@ struct TcCfg {
     static_assert(S >= 2, "shared memory too small for a double-buffered ring");
     static_assert(Q_BYTES % 1024 == 0 && P_BYTES % 1024 == 0 && STAGE_BYTES % 1024 == 0, "");
 };
+
+// Maximum over the warp's 32 lanes of each of v[0..NH): NH-1 shuffles halve the values per lane,
+// then 5 - log2(NH) butterflies finish.  Lane l ends with, in v[0], the result for head
+// sum_s bit_s(l) * NH / 2^(s+1) (the bit-reversed low bits of l).
+template <int NH, int LOG2NH>
+__device__ __forceinline__ void warp_max_transpose(float (&v)[NH], int lane) {
+#pragma unroll
+    for (int s = 0; s < LOG2NH; ++s) {
+        const int half = NH >> (s + 1);
+        const bool upper = (lane >> s) & 1;
+#pragma unroll
+        for (int j = 0; j < NH / 2; ++j) {
+            if (j < half) {
+                const float send = upper ? v[j] : v[j + half];
+                const float keep = upper ? v[j + half] : v[j];
+                v[j] = fmaxf(keep, __shfl_xor_sync(kFullMask, send, 1 << s));
+            }
+        }
+    }
+#pragma unroll
+    for (int off = 1 << LOG2NH; off < 32; off <<= 1) v[0] = fmaxf(v[0], __shfl_xor_sync(kFullMask, v[0], off));
+}
+
+template <int NH, int LOG2NH>
+__device__ __forceinline__ int transpose_head(int lane) {
+    int h = 0;
+#pragma unroll
+    for (int s = 0; s < LOG2NH; ++s) h += ((lane >> s) & 1) * (NH >> (s + 1));
+    return h;
+}
 
 // Add a byte offset to a shared-memory descriptor's start address (bits 0-13, 16-byte units).
 // Shared addresses stay below 2^18, so the field cannot carry into the next one.
@@ -239,11 +275,11 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (lane == 0) {
             // K tile and Q: K-major (rows / heads by d), 8-row groups 1024 B apart.
             // V^T: MN-major (d by rows): the two 64-column blocks T*128 B apart.
-            // P^T: K-major (2*RP rows by tile rows).
+            // P^T: MN-major (2*RP values per tile row), 8-row groups 8*P_ROWB apart.
             const uint64_t dk0 = sdesc_sw128(smem_u32(st_base), 16, 1024);
             const uint64_t dv0 = sdesc_sw128(smem_u32(st_base + C::TILE_BYTES), T * 128, 1024);
             const uint64_t dq0 = sdesc_sw128(smem_u32(q_base), 16, 1024);
-            const uint64_t dp0 = sdesc_sw128(smem_u32(p_base), 16, 1024);
+            const uint64_t dp0 = sdesc_swz(smem_u32(p_base), C::P_ATOMB, 8 * C::P_ROWB, C::P_LAYOUT);
             SegmentWalker w;
             w.init(p, cr);
             Segment sg;
@@ -295,9 +331,8 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         // N = 2*RP product.
 #pragma unroll
                         for (int kk = 0; kk < T / 16; ++kk) {
-                            const uint32_t off_p = (kk >> 2) * 2 * RP * 128 + (kk & 3) * 32;
                             umma_bf16(tmem + C::O_COL + j2 * C::O_COL, desc_add(dv, kk * 2048),
-                                      desc_add(dp, off_p), C::IDESC_PV, kk > 0 ? 1u : 0u);
+                                      desc_add(dp, kk * 16 * C::P_ROWB), C::IDESC_PV, kk > 0 ? 1u : 0u);
                         }
                         umma_commit(&sm->o_full[j2]);
                         umma_commit(&sm->kv_empty[pv_t % S]);
@@ -327,10 +362,6 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const uint32_t lane_addr = static_cast<uint32_t>(q4 * 32) << 16;
         // Output column (of d) this thread accumulates: O^T row in TMEM.
         const int dcol = (D == 128) ? row : (lane < 16 ? q4 * 16 + lane : -1);
-        // Where this thread's row lands in P^T: column `row` of every head row.
-        const int col = row & 63;
-        const int chunk = col >> 3;
-        const int within = (col & 7) * 2;
         SegmentWalker w;
         w.init(p, cr);
         Segment sg;
@@ -391,19 +422,14 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                 for (int h = 0; h < NH; ++h)
                     x[h] = valid ? __uint_as_float(sr[h]) * p.scale_log2 : -INFINITY;
-                // Per-head maximum over the warp's 32 rows: interleaved butterflies.
-                float wm[NH];
+                // Per-head maximum over the warp's 32 rows.
+                {
+                    float wm[NH];
 #pragma unroll
-                for (int h = 0; h < NH; ++h) wm[h] = x[h];
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1) {
-#pragma unroll
-                    for (int h = 0; h < NH; ++h) wm[h] = fmaxf(wm[h], __shfl_xor_sync(kFullMask, wm[h], off));
-                }
-                if (lane == 0) {
-                    float *dst = reinterpret_cast<float *>(&sm->wmax[j2][q4][0]);
-#pragma unroll
-                    for (int h = 0; h < NH; ++h) dst[h] = wm[h];
+                    for (int h = 0; h < NH; ++h) wm[h] = x[h];
+                    warp_max_transpose<NH, C::LOG2NH>(wm, lane);
+                    if (lane < NH)
+                        reinterpret_cast<float *>(&sm->wmax[j2][q4][0])[transpose_head<NH, C::LOG2NH>(lane)] = wm[0];
                 }
                 if (named_bar_any(1, 128, bad)) {
                     ok = false;
@@ -446,28 +472,44 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     named_bar_sync(1, 128);  // every thread of the group arrives here
                 }
 
-                // P^T as bf16 high and low parts (P = hi + lo to ~16 bits), K-major with
-                // 128-byte swizzle: row h holds head h's high parts, row RP + h its low parts,
-                // tile row r is column r (64 columns per 128-byte row, two column blocks).
-                uint8_t *pb = p_base + j2 * C::P_BYTES + (row >> 6) * 2 * RP * 128;
+                // P = hi + lo in bf16 (~16 significant bits).  This thread's tile row is K row
+                // `row` of the MN-major P^T: high parts at values [0, RP), low parts at [RP, 2RP),
+                // written as 16-byte chunks of 8 heads.
+                {
+                    uint8_t *prow = p_base + j2 * C::P_BYTES + row * C::P_ROWB;
+                    const int swz = C::P_ROWB == 128 ? (row & 7) : ((row >> 1) & 3);
+                    constexpr int HALF_VALS = C::P_ROWB / 2;  // bf16 values per atom row
 #pragma unroll
-                for (int h = 0; h < NH; ++h) {
-                    float m_h, a_h;
-                    if constexpr (C::REG_STATE) {
-                        m_h = m_run[h];
-                        a_h = alpha[h];
-                    } else {
-                        m_h = sm->mcur[j2][h];
-                        a_h = sm->alpha[j2][h];
+                    for (int h = 0; h < NH; ++h) {
+                        float m_h, a_h;
+                        if constexpr (C::REG_STATE) {
+                            m_h = m_run[h];
+                            a_h = alpha[h];
+                        } else {
+                            m_h = sm->mcur[j2][h];
+                            a_h = sm->alpha[j2][h];
+                        }
+                        x[h] = ex2_approx(x[h] - m_h);  // x now holds p
+                        l[h] = l[h] * a_h + x[h];
                     }
-                    const float pr = ex2_approx(x[h] - m_h);
-                    const __nv_bfloat16 hi = __float2bfloat16_rn(pr);
-                    const __nv_bfloat16 lo = __float2bfloat16_rn(pr - __bfloat162float(hi));
-                    l[h] = l[h] * a_h + pr;
-                    if (h < nh) {
-                        uint8_t *dst = pb + h * 128 + ((chunk ^ (h & 7)) << 4) + within;
-                        *reinterpret_cast<__nv_bfloat16 *>(dst) = hi;
-                        *reinterpret_cast<__nv_bfloat16 *>(dst + RP * 128) = lo;
+#pragma unroll
+                    for (int c8 = 0; c8 < (NH + 7) / 8; ++c8) {
+                        uint32_t hw[4], lw[4];
+#pragma unroll
+                        for (int w2 = 0; w2 < 4; ++w2) {
+                            const int h = c8 * 8 + 2 * w2;
+                            const float a = h < NH ? x[h] : 0.f;
+                            const float b = h + 1 < NH ? x[h + 1] : 0.f;
+                            const __nv_bfloat162 hi = __floats2bfloat162_rn(a, b);
+                            const __nv_bfloat162 lo = __floats2bfloat162_rn(a - __low2float(hi), b - __high2float(hi));
+                            hw[w2] = *reinterpret_cast<const uint32_t *>(&hi);
+                            lw[w2] = *reinterpret_cast<const uint32_t *>(&lo);
+                        }
+                        const int eh = c8 * 8, el = RP + c8 * 8;
+                        *reinterpret_cast<uint4 *>(prow + (eh / HALF_VALS) * C::P_ATOMB + ((((eh % HALF_VALS) >> 3) ^ swz) << 4)) =
+                            make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                        *reinterpret_cast<uint4 *>(prow + (el / HALF_VALS) * C::P_ATOMB + ((((el % HALF_VALS) >> 3) ^ swz) << 4)) =
+                            make_uint4(lw[0], lw[1], lw[2], lw[3]);
                     }
                 }
                 fence_proxy_async_smem();

@@ -199,15 +199,21 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t *r) {
 //   bits 32-45  stride-dimension byte offset >> 4
 //   bits 46-47  descriptor version (1 on sm_100)
 //   bits 61-63  layout: 2 = 128-byte swizzle
-__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_bytes,
-                                                uint32_t sbo_bytes) {
+//   (layout 4 = 64-byte swizzle, used by sdesc_sw64)
+__device__ __forceinline__ uint64_t sdesc_swz(uint32_t saddr, uint32_t lbo_bytes,
+                                              uint32_t sbo_bytes, uint32_t layout) {
     uint64_t d = 0;
     d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
     d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
     d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
     d |= static_cast<uint64_t>(1) << 46;
-    d |= static_cast<uint64_t>(2) << 61;
+    d |= static_cast<uint64_t>(layout) << 61;
     return d;
+}
+
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_bytes,
+                                                uint32_t sbo_bytes) {
+    return sdesc_swz(saddr, lbo_bytes, sbo_bytes, 2);
 }
 
 // UMMA instruction descriptor for kind::f16 with bf16 A and B, fp32 D.
