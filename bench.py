@@ -183,7 +183,11 @@ def bench_ours(args, rank, world, local):
     def step(i, lens_row, qq=q, kk=kn, vv=vn):
         kc, vc = caches[i & 1]
         gqa.kv_append(kk, vv, kc, vc, lens_row, status=status)
-        gqa.decode(qq, kc, vc, lens_row, x["scale"], out=out, workspace=ws, status=status)
+        if w.window > 0:
+            gqa.decode_window(qq, kc, vc, lens_row, w.window, x["scale"], out=out, workspace=ws,
+                              status=status)
+        else:
+            gqa.decode(qq, kc, vc, lens_row, x["scale"], out=out, workspace=ws, status=status)
 
     # correctness guard before timing
     lens_chk = lens0.clone()
@@ -312,6 +316,7 @@ def bench_ours(args, rank, world, local):
             "config": {
                 "workload": w.name, "B": w.B, "H_q": w.H_q, "H_kv": w.H_kv, "d": w.d,
                 "L_max": w.L_max, "seq_len": lengths[0] if w.length else "ragged",
+                "window": w.window or None,
                 "sum_seq_lens": int(sum(lengths)), "kv_dtype": str(w.dtype).replace("torch.", ""),
                 "accumulate": "f32", "ideal_kv_bytes_per_step": ideal,
                 "parallelism": f"replicas x{world}",
@@ -364,7 +369,10 @@ def cpu_baseline(w, x, budget_s, steps=None):
         lens = xb["seq_lens_pre"].numpy().copy()
         ts = time.perf_counter()
         o.kv_append(xb["k_new"].double().numpy(), xb["v_new"].double().numpy(), kc, vc, lens)
-        o.decode(q, kc, vc, lens, x["scale"])
+        if w.window > 0:
+            o.decode_window(q, kc, vc, lens, w.window, x["scale"])
+        else:
+            o.decode(q, kc, vc, lens, x["scale"])
         done.append(time.perf_counter() - ts)
         nbytes += inputs.ideal_kv_bytes(w, lens.tolist())
         b = (b + 1) % B
@@ -395,7 +403,11 @@ def profile_run(args, local):
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     for i in range(args.warmup + args.steps):
         gqa.kv_append(kn, vn, kc, vc, lens_rows[i], status=status)
-        gqa.decode(q, kc, vc, lens_rows[i], x["scale"], out=out, workspace=ws, status=status)
+        if w.window > 0:
+            gqa.decode_window(q, kc, vc, lens_rows[i], w.window, x["scale"], out=out,
+                              workspace=ws, status=status)
+        else:
+            gqa.decode(q, kc, vc, lens_rows[i], x["scale"], out=out, workspace=ws, status=status)
     torch.cuda.synchronize()
     st = int(status.item())
     assert st == 0, f"device status {st}"

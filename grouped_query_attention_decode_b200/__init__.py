@@ -25,10 +25,12 @@ STATUS_APPEND_OVERFLOW = 1
 STATUS_SEQLEN_RANGE = 2
 STATUS_WAIT_TIMEOUT = 4
 STATUS_INTERNAL = 8
+STATUS_PAGE_RANGE = 16
 
 # C-ABI symbols declared in include/gqa.h
 EXPORTED = ("gqa_kv_append", "gqa_decode_workspace_size", "gqa_decode", "gqa_status_string",
-            "gqa_set_wait_timeout_ns", "gqa_profile_events", "gqa_decode_noalloc")
+            "gqa_set_wait_timeout_ns", "gqa_profile_events", "gqa_decode_noalloc",
+            "gqa_decode_window", "gqa_kv_append_paged", "gqa_decode_paged")
 
 
 class GQAError(RuntimeError):
@@ -60,6 +62,15 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gqa_decode.argtypes = [vp, vp, vp, i32p, c_int, c_int, c_int, c_int, c_int,
                                ctypes.c_float, c_int, vp, vp, c_size, i32p, vp]
     lib.gqa_decode.restype = c_int
+    lib.gqa_decode_window.argtypes = [vp, vp, vp, i32p, c_int, c_int, c_int, c_int, c_int, c_int,
+                                      ctypes.c_float, c_int, vp, vp, c_size, i32p, vp]
+    lib.gqa_decode_window.restype = c_int
+    lib.gqa_kv_append_paged.argtypes = [vp, vp, vp, vp, i32p, c_int, i32p, c_int, c_int, c_int,
+                                        c_int, c_int, c_int, i32p, vp]
+    lib.gqa_kv_append_paged.restype = c_int
+    lib.gqa_decode_paged.argtypes = [vp, vp, vp, i32p, c_int, i32p, c_int, c_int, c_int, c_int,
+                                     c_int, c_int, ctypes.c_float, c_int, vp, vp, c_size, i32p, vp]
+    lib.gqa_decode_paged.restype = c_int
     lib.gqa_decode_noalloc.argtypes = [vp, vp, vp, i32p, c_int, c_int, c_int, c_int, c_int,
                                        ctypes.c_float, c_int, vp, i32p, vp]
     lib.gqa_decode_noalloc.restype = c_int
@@ -134,6 +145,50 @@ def decode(q, k_cache, v_cache, seq_lens, scale: float, out=None, workspace=None
         _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens), B, H_q, H_kv, d, L_max,
         float(scale), _dtype(k_cache), _ptr(out), _ptr(workspace), workspace.numel(),
         _ptr(status), _stream(stream)))
+    return out
+
+
+def decode_window(q, k_cache, v_cache, seq_lens, window: int, scale: float, out=None,
+                  workspace=None, status=None, stream=None) -> torch.Tensor:
+    """gqa_decode_window: each sequence attends only its last ``window`` cached rows."""
+    B, H_q, d = q.shape
+    _, L_max, H_kv, _ = k_cache.shape
+    if out is None:
+        out = torch.empty((B, H_q, d), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(B, H_q, H_kv, d, k_cache.dtype, device=q.device)
+    _check(load_library().gqa_decode_window(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens), B, H_q, H_kv, d, L_max,
+        int(window), float(scale), _dtype(k_cache), _ptr(out), _ptr(workspace),
+        workspace.numel(), _ptr(status), _stream(stream)))
+    return out
+
+
+def kv_append_paged(k_new, v_new, k_pool, v_pool, block_table, seq_lens, status=None,
+                    stream=None) -> None:
+    """gqa_kv_append_paged: pools [n_pages, page_size, H_kv, d], block_table [B, max_pages]."""
+    n_pages, page_size, H_kv, d = k_pool.shape
+    B, max_pages = block_table.shape
+    _check(load_library().gqa_kv_append_paged(
+        _ptr(k_new), _ptr(v_new), _ptr(k_pool), _ptr(v_pool), _ptr(block_table), max_pages,
+        _ptr(seq_lens), B, H_kv, d, page_size, n_pages, _dtype(k_pool), _ptr(status),
+        _stream(stream)))
+
+
+def decode_paged(q, k_pool, v_pool, block_table, seq_lens, scale: float, out=None,
+                 workspace=None, status=None, stream=None) -> torch.Tensor:
+    """gqa_decode_paged: the decode over a paged cache."""
+    B, H_q, d = q.shape
+    n_pages, page_size, H_kv, _ = k_pool.shape
+    _, max_pages = block_table.shape
+    if out is None:
+        out = torch.empty((B, H_q, d), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(B, H_q, H_kv, d, k_pool.dtype, device=q.device)
+    _check(load_library().gqa_decode_paged(
+        _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(block_table), max_pages, _ptr(seq_lens), B,
+        H_q, H_kv, d, page_size, n_pages, float(scale), _dtype(k_pool), _ptr(out),
+        _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream)))
     return out
 
 

@@ -156,10 +156,18 @@ extern "C" size_t gqa_decode_workspace_size(int B, int H_q, int H_kv, int d, gqa
     return geometry(B, H_q, H_kv, d, sms).bytes;
 }
 
-extern "C" int gqa_decode(const void *q, const void *k_cache, const void *v_cache,
-                          const int32_t *seq_lens, int B, int H_q, int H_kv, int d, int L_max,
-                          float scale, gqa_dtype_t dtype, float *out, void *workspace,
-                          size_t workspace_bytes, int32_t *status, cudaStream_t stream) {
+namespace {
+
+// Paged cache description for decode_impl (block_table == nullptr: contiguous caches).
+struct PagedArgs {
+    const int32_t *block_table = nullptr;
+    int max_pages = 0, page_size = 0, n_pages = 0;
+};
+
+int decode_impl(const void *q, const void *k_cache, const void *v_cache, const int32_t *seq_lens,
+                int B, int H_q, int H_kv, int d, int L_max, int window, float scale,
+                gqa_dtype_t dtype, float *out, void *workspace, size_t workspace_bytes,
+                int32_t *status, cudaStream_t stream, const PagedArgs &pg = PagedArgs()) {
     if (!q || !k_cache || !v_cache || !seq_lens || !out) return GQA_ERR_NULL;
     const int rc = check_shape(B, H_q, H_kv, d, L_max, dtype);
     if (rc != GQA_OK) return rc;
@@ -189,9 +197,15 @@ extern "C" int gqa_decode(const void *q, const void *k_cache, const void *v_cach
     p.HB = g.HB;
     p.UB = g.UB;
     p.T = dtype == GQA_DTYPE_BF16 ? 128 : 64;
+    p.window = window;
+    p.block_table = pg.block_table;
+    p.max_pages = pg.max_pages;
+    p.page_size = pg.page_size;
+    p.n_pages = pg.n_pages;
     // One persistent CTA per SM, but never more CTAs than the largest possible tile count
     // (the workspace is sized for one per SM, which bounds this).
-    const long long max_tiles = g.units * ((static_cast<long long>(L_max) + p.T - 1) / p.T);
+    const long long span = (window > 0 && window < L_max) ? window : L_max;
+    const long long max_tiles = g.units * ((span + p.T - 1) / p.T);
     p.G = max_tiles < sms ? static_cast<int>(max_tiles) : sms;
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     p.wait_ns = g_wait_ns.load();
@@ -205,11 +219,15 @@ extern "C" int gqa_decode(const void *q, const void *k_cache, const void *v_cach
         const int rp = tc_q_box_rows(g.RB);
         if (encode_fn() == nullptr) return GQA_ERR_CUDA;
         TmaMaps maps;
+        // The cache as (d, H_kv, rows, sequences) -- or, paged, (d, H_kv, page_size, n_pages).
+        const int rows_dim = pg.block_table ? pg.page_size : L_max;
+        const int outer_dim = pg.block_table ? pg.n_pages : B;
+        const int box = pg.block_table ? (pg.page_size < 128 ? pg.page_size : 128) : 128;
         if (!encode_q_map(&maps.q, q, B, H_q, d, rp) ||
-            !encode_cache_map(&maps.k, k_cache, B, H_kv, d, L_max, 128) ||
-            !encode_cache_map(&maps.k8, k_cache, B, H_kv, d, L_max, 8) ||
-            !encode_cache_map(&maps.v, v_cache, B, H_kv, d, L_max, 128) ||
-            !encode_cache_map(&maps.v8, v_cache, B, H_kv, d, L_max, 8))
+            !encode_cache_map(&maps.k, k_cache, outer_dim, H_kv, d, rows_dim, box) ||
+            !encode_cache_map(&maps.k8, k_cache, outer_dim, H_kv, d, rows_dim, 8) ||
+            !encode_cache_map(&maps.v, v_cache, outer_dim, H_kv, d, rows_dim, box) ||
+            !encode_cache_map(&maps.v8, v_cache, outer_dim, H_kv, d, rows_dim, 8))
             return GQA_ERR_SHAPE;
         if (profile && cudaEventRecord(ev0, stream) != cudaSuccess) return GQA_ERR_CUDA;
         res = launch_split_tc(maps, p, stream);
@@ -221,6 +239,71 @@ extern "C" int gqa_decode(const void *q, const void *k_cache, const void *v_cach
     if (res != GQA_OK) return res;
     if (profile && cudaEventRecord(ev1, stream) != cudaSuccess) return GQA_ERR_CUDA;
     return launch_combine(p, stream);
+}
+
+}  // namespace
+
+extern "C" int gqa_decode(const void *q, const void *k_cache, const void *v_cache,
+                          const int32_t *seq_lens, int B, int H_q, int H_kv, int d, int L_max,
+                          float scale, gqa_dtype_t dtype, float *out, void *workspace,
+                          size_t workspace_bytes, int32_t *status, cudaStream_t stream) {
+    return decode_impl(q, k_cache, v_cache, seq_lens, B, H_q, H_kv, d, L_max, 0, scale, dtype,
+                       out, workspace, workspace_bytes, status, stream);
+}
+
+extern "C" int gqa_kv_append_paged(const void *k_new, const void *v_new, void *k_pool,
+                                   void *v_pool, const int32_t *block_table, int max_pages,
+                                   int32_t *seq_lens, int B, int H_kv, int d, int page_size,
+                                   int n_pages, gqa_dtype_t dtype, int32_t *status,
+                                   cudaStream_t stream) {
+    if (!k_new || !v_new || !k_pool || !v_pool || !block_table || !seq_lens) return GQA_ERR_NULL;
+    if (dtype != GQA_DTYPE_F32 && dtype != GQA_DTYPE_BF16) return GQA_ERR_UNSUPPORTED_DTYPE;
+    if (B <= 0 || H_kv <= 0 || max_pages <= 0 || n_pages <= 0 || page_size <= 0 ||
+        page_size % 8 != 0 || static_cast<long long>(max_pages) * page_size > (1ll << 30) ||
+        static_cast<long long>(B) * H_kv > (1ll << 30))
+        return GQA_ERR_SHAPE;
+    if (d != 64 && d != 128) return GQA_ERR_UNSUPPORTED_DIM;
+    if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(k_pool, 16) ||
+        !aligned(v_pool, 16) || !aligned(seq_lens, 4) || !aligned(block_table, 4) ||
+        (status && !aligned(status, 4)))
+        return GQA_ERR_ALIGNMENT;
+    int dev = 0;
+    if (current_sm_count(&dev) <= 0) return GQA_ERR_NO_DEVICE;
+    const int row_bytes = d * (dtype == GQA_DTYPE_BF16 ? 2 : 4);
+    return launch_append_paged(k_new, v_new, k_pool, v_pool, block_table, max_pages, seq_lens, B,
+                               H_kv, row_bytes, page_size, n_pages, status, stream);
+}
+
+extern "C" int gqa_decode_paged(const void *q, const void *k_pool, const void *v_pool,
+                                const int32_t *block_table, int max_pages,
+                                const int32_t *seq_lens, int B, int H_q, int H_kv, int d,
+                                int page_size, int n_pages, float scale, gqa_dtype_t dtype,
+                                float *out, void *workspace, size_t workspace_bytes,
+                                int32_t *status, cudaStream_t stream) {
+    if (!block_table) return GQA_ERR_NULL;
+    if (!aligned(block_table, 4)) return GQA_ERR_ALIGNMENT;
+    if (max_pages <= 0 || n_pages <= 0 || page_size <= 0 || page_size % 8 != 0 ||
+        static_cast<long long>(max_pages) * page_size > (1ll << 30))
+        return GQA_ERR_SHAPE;
+    // a 128-row tile must lie in one page or cover whole pages
+    if (dtype == GQA_DTYPE_BF16 && 128 % page_size != 0 && page_size % 128 != 0) return GQA_ERR_SHAPE;
+    PagedArgs pg;
+    pg.block_table = block_table;
+    pg.max_pages = max_pages;
+    pg.page_size = page_size;
+    pg.n_pages = n_pages;
+    return decode_impl(q, k_pool, v_pool, seq_lens, B, H_q, H_kv, d, max_pages * page_size, 0,
+                       scale, dtype, out, workspace, workspace_bytes, status, stream, pg);
+}
+
+extern "C" int gqa_decode_window(const void *q, const void *k_cache, const void *v_cache,
+                                 const int32_t *seq_lens, int B, int H_q, int H_kv, int d,
+                                 int L_max, int window, float scale, gqa_dtype_t dtype,
+                                 float *out, void *workspace, size_t workspace_bytes,
+                                 int32_t *status, cudaStream_t stream) {
+    if (window <= 0) return GQA_ERR_SHAPE;
+    return decode_impl(q, k_cache, v_cache, seq_lens, B, H_q, H_kv, d, L_max, window, scale,
+                       dtype, out, workspace, workspace_bytes, status, stream);
 }
 
 extern "C" const char *gqa_status_string(int code) {

@@ -42,7 +42,7 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const DecodePa
     float *o = p.out + (static_cast<long long>(b) * p.H_q + h0) * d;
     const long long *hdr = reinterpret_cast<const long long *>(p.ws);
     const int n = valid_len(p.seq_lens[b], p.L_max);
-    const int nt = tiles_of(n, p.T);
+    const int nt = seq_tiles(n, p);
     if (nt == 0) {
         for (int idx = first + threadIdx.x; idx < last; idx += blockDim.x) o[idx] = 0.f;
         return;

@@ -82,15 +82,26 @@ split_f32_kernel(const float *__restrict__ q, const float *__restrict__ kc,
         for (int k = 0; k < ACC; ++k) acc[k] = 0.f;
         __syncthreads();
         for (int jj = 0; jj < sg.len; ++jj) {
-            const int row0 = (sg.j0 + jj) * T;
+            const int row0 = sg.first + (sg.j0 + jj) * T;
             const int rows = min(T, sg.n - row0);
-            const long long base = ((static_cast<long long>(sg.b) * p.L_max + row0) * p.H_kv + sg.kvh) * D;
-            const long long rstride = static_cast<long long>(p.H_kv) * D;
             for (int idx = tid; idx < rows * (D / 4); idx += 256) {
                 const int t = idx / (D / 4);
                 const int c4 = idx - t * (D / 4);
-                const float4 kv = *reinterpret_cast<const float4 *>(kc + base + t * rstride + 4 * c4);
-                const float4 vv = *reinterpret_cast<const float4 *>(vc + base + t * rstride + 4 * c4);
+                // element offset of cached row row0 + t of this key/value head
+                long long off;
+                if (p.block_table != nullptr) {
+                    const int lr = row0 + t;
+                    int pg = p.block_table[static_cast<long long>(sg.b) * p.max_pages + lr / p.page_size];
+                    if (pg < 0 || pg >= p.n_pages) {
+                        if (p.status != nullptr) atomicOr(p.status, GQA_STATUS_PAGE_RANGE);
+                        pg = 0;
+                    }
+                    off = ((static_cast<long long>(pg) * p.page_size + lr % p.page_size) * p.H_kv + sg.kvh) * D;
+                } else {
+                    off = ((static_cast<long long>(sg.b) * p.L_max + row0 + t) * p.H_kv + sg.kvh) * D;
+                }
+                const float4 kv = *reinterpret_cast<const float4 *>(kc + off + 4 * c4);
+                const float4 vv = *reinterpret_cast<const float4 *>(vc + off + 4 * c4);
                 *reinterpret_cast<float4 *>(ks + t * KP + 4 * c4) = kv;
                 *reinterpret_cast<float4 *>(vs + t * D + 4 * c4) = vv;
             }

@@ -15,10 +15,11 @@
 // rounding residual) side by side, summed when the tile is read back, so it carries ~16
 // significant bits rather than 8.  NH is the group's head count rounded up to a power of two
 // (1..64) and RP = max(16, NH) the UMMA N; padded heads are computed and ignored.
-// Roles (192 threads):
+// Roles (64 + 128 * NWG threads):
 //   warp 0       TMA producer (q of each unit, K/V tiles); also owns the tensor memory
 //   warp 1       UMMA issuer (one elected thread, event loop)
-//   warps 2..5   softmax / accumulation / epilogue (128 threads)
+//   warps 2..    NWG softmax / accumulation / epilogue warpgroups of 128 threads, each owning
+//                a slice of the group's query heads (one warpgroup up to 16 heads)
 // Every wait is bounded; on a timeout the CTA drains its in-flight copies and UMMAs, frees
 // its tensor memory, sets GQA_STATUS_WAIT_TIMEOUT and returns.
 #include <cstdint>
@@ -52,11 +53,13 @@ struct TcCfg {
     static constexpr int TMEM_COLS = 6 * RP <= 128 ? 128 : (6 * RP <= 256 ? 256 : 512);
     static constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, RP, false, false);
     static constexpr uint32_t IDESC_PV = idesc_bf16_f32(D, 2 * RP, true, true);
-    // Running max and rescale factors live in registers up to 32 heads; with 64 heads they go
-    // through shared memory to keep the softmax threads under the register limit.
-    static constexpr bool REG_STATE = NH <= 32;
-    static constexpr int NH4 = (NH + 3) / 4;
-    static constexpr int LOG2NH = NH >= 64 ? 6 : NH >= 32 ? 5 : NH >= 16 ? 4 : NH >= 8 ? 3 : NH >= 4 ? 2 : NH >= 2 ? 1 : 0;
+    // Softmax warpgroups: one for up to 16 heads, else one per 16 heads (heads are
+    // independent, so the groups split them and never exchange data).
+    static constexpr int NWG = NH >= 32 ? NH / 16 : 1;
+    static constexpr int NHW = NH / NWG;              // heads per warpgroup
+    static constexpr int THREADS = 64 + 128 * NWG;
+    static constexpr int NHW4 = (NHW + 3) / 4;
+    static constexpr int LOG2NHW = NHW >= 16 ? 4 : NHW >= 8 ? 3 : NHW >= 4 ? 2 : NHW >= 2 ? 1 : 0;
 
     struct Small {
         uint64_t kv_full[8], kv_empty[8];
@@ -68,10 +71,8 @@ struct TcCfg {
         int b0;
         int pad_;
         long long begin, end, off0;
-        float4 wmax[2][4][NH4];  // per tile parity, warp: the warp's per-head maxima
-        float mcur[2][NH];       // 64-head path only
-        float alpha[2][NH];      // 64-head path only
-        float lsum[4][NH];
+        float4 wmax[NWG][2][4][NHW4];  // per group, tile parity, warp: per-head warp maxima
+        float lsum[NWG][4][NHW];
     };
 
     static constexpr int SMEM_LIMIT = 232448;
@@ -122,8 +123,8 @@ __device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t bytes) {
     return desc + static_cast<uint64_t>(bytes >> 4);
 }
 
-template <int D, int NH>
-__global__ void __launch_bounds__(192, 1)
+template <int D, int NH, bool PAGED>
+__global__ void __launch_bounds__(TcCfg<D, NH>::THREADS, 1)
 split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_k8, const __grid_constant__ CUtensorMap tm_v,
                 const __grid_constant__ CUtensorMap tm_v8, const DecodeParams p) {
@@ -154,10 +155,10 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mbar_init(&sm->q_full[j], 1);
             mbar_init(&sm->q_empty[j], 1);
             mbar_init(&sm->s_full[j], 1);
-            mbar_init(&sm->s_empty[j], 4);
-            mbar_init(&sm->p_full[j], 4);
+            mbar_init(&sm->s_empty[j], 4 * C::NWG);
+            mbar_init(&sm->p_full[j], 4 * C::NWG);
             mbar_init(&sm->o_full[j], 1);
-            mbar_init(&sm->o_empty[j], 4);
+            mbar_init(&sm->o_empty[j], 4 * C::NWG);
         }
         mbar_init(&sm->mma_done, 1);
         sm->abort = 0;
@@ -230,15 +231,52 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 ++sidx;
                 for (int jj = 0; jj < sg.len; ++jj) {
                     const int st = i % S;
+                    const int row0 = sg.first + (sg.j0 + jj) * T;
+                    const int rows = min(T, sg.n - row0);
+                    // Paged cache: page of each box of the tile (boxes of min(page_size, T) rows,
+                    // or 8 rows for a partial tile), loaded before the wait for a free stage so
+                    // that the lookups overlap it.
+                    int page[16];
+                    int boxr = T;
+                    if constexpr (PAGED) {
+                        boxr = rows == T ? min(p.page_size, T) : 8;
+                        const int nbox = rows == T ? T / boxr : (rows + 7) >> 3;
+                        const int32_t *bt = p.block_table + static_cast<long long>(sg.b) * p.max_pages;
+#pragma unroll
+                        for (int x = 0; x < 16; ++x) {
+                            if (x < nbox) {
+                                int pg = bt[(row0 + x * boxr) / p.page_size];
+                                if (pg < 0 || pg >= p.n_pages) {
+                                    if (p.status != nullptr) atomicOr(p.status, GQA_STATUS_PAGE_RANGE);
+                                    pg = 0;
+                                }
+                                page[x] = pg;
+                            }
+                        }
+                    }
                     if (i >= S && !wait_bounded(&sm->kv_empty[st], ((i / S) - 1) & 1, abort_flag, budget)) {
                         ok = false;
                         break;
                     }
-                    const int row0 = (sg.j0 + jj) * T;
-                    const int rows = min(T, sg.n - row0);
                     uint8_t *kdst = st_base + st * C::STAGE_BYTES;
                     uint8_t *vdst = kdst + C::TILE_BYTES;
-                    if (rows == T) {
+                    if constexpr (PAGED) {
+                        const int nbox = rows == T ? T / boxr : (rows + 7) >> 3;
+                        const CUtensorMap *mk = rows == T ? &tm_k : &tm_k8;
+                        const CUtensorMap *mv = rows == T ? &tm_v : &tm_v8;
+                        mbar_arrive_expect_tx(&sm->kv_full[st], 2 * C::KB * nbox * boxr * 128);
+#pragma unroll
+                        for (int x = 0; x < 16; ++x) {
+                            if (x < nbox) {
+                                const int pr = (row0 + x * boxr) % p.page_size;
+#pragma unroll
+                                for (int kb = 0; kb < C::KB; ++kb) {
+                                    tma_load_4d(kdst + kb * T * 128 + x * boxr * 128, mk, &sm->kv_full[st], kb * 64, sg.kvh, pr, page[x], pol);
+                                    tma_load_4d(vdst + kb * T * 128 + x * boxr * 128, mv, &sm->kv_full[st], kb * 64, sg.kvh, pr, page[x], pol);
+                                }
+                            }
+                        }
+                    } else if (rows == T) {
                         mbar_arrive_expect_tx(&sm->kv_full[st], C::STAGE_BYTES);
 #pragma unroll
                         for (int kb = 0; kb < C::KB; ++kb) {
@@ -356,9 +394,17 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
     } else {
         // ------------------------------------------------------------------ softmax warps
-        const int q4 = warp & 3;               // TMEM lane quadrant this warp may access
-        const int row = q4 * 32 + lane;        // tile row of S^T this thread owns
-        const int wg_tid = threadIdx.x - 64;   // 0..127
+        // NWG warpgroups of four warps; warpgroup g owns query heads [g*NHW, (g+1)*NHW) of the
+        // unit.  Heads are independent, so the groups never exchange data: each has its own
+        // named barrier (1 + g) and its own per-head state.
+        constexpr int NHW = C::NHW;
+        constexpr int SCOLS = C::NWG == 1 ? RP : NHW;  // S^T columns this group loads
+        const int wg = (warp - 2) >> 2;
+        const int hbase = wg * NHW;
+        const uint32_t bar_id = 1 + wg;
+        const int q4 = warp & 3;                 // TMEM lane quadrant this warp may access
+        const int row = q4 * 32 + lane;          // tile row of S^T this thread owns
+        const int sm_tid = threadIdx.x - 64;     // 0 .. 128*NWG-1
         const uint32_t lane_addr = static_cast<uint32_t>(q4 * 32) << 16;
         // Output column (of d) this thread accumulates: O^T row in TMEM.
         const int dcol = (D == 128) ? row : (lane < 16 ? q4 * 16 + lane : -1);
@@ -367,34 +413,28 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         Segment sg;
         int i = 0;
         bool ok = true;
-        float O[NH];
-        float l[NH];
-        float m_run[C::REG_STATE ? NH : 1];
-        float alpha[C::REG_STATE ? NH : 1];
+        float O[NHW], l[NHW], m_run[NHW], alpha[NHW];
         while (ok && w.next(sg)) {
             const int nh = min(p.RB, p.r - sg.hb * p.RB);
+            const int nhw = min(NHW, max(0, nh - hbase));  // this group's real heads
 #pragma unroll
-            for (int h = 0; h < NH; ++h) {
+            for (int h = 0; h < NHW; ++h) {
                 O[h] = 0.f;
                 l[h] = 0.f;
+                m_run[h] = -INFINITY;
             }
-            if constexpr (C::REG_STATE) {
-#pragma unroll
-                for (int h = 0; h < NH; ++h) m_run[h] = -INFINITY;
-            }
-            int j2 = 0;
             // A failed wait sets `bad`; the threads then agree at the next named barrier
             // (named_bar_any) and leave together, so no warp is left waiting at a barrier.
             bool bad = false;
             for (int jj = 0; jj < sg.len; ++jj, ++i) {
-                j2 = i & 1;
-                const int rows = min(T, sg.n - (sg.j0 + jj) * T);
+                const int j2 = i & 1;
+                const int rows = min(T, sg.n - sg.first - (sg.j0 + jj) * T);
                 if (rows < T && !bad && wait_bounded(&sm->kv_full[i % S], (i / S) & 1, abort_flag, budget)) {
                     // Rows past n: zero V in shared memory so that 0-weight rows add exactly 0
                     // (stale or unread data there may hold NaN or Inf).
                     uint8_t *vbase = st_base + (i % S) * C::STAGE_BYTES + C::TILE_BYTES;
                     const int nchunks = (T - rows) * 8;  // 16-byte chunks per column block
-                    for (int c = wg_tid; c < nchunks * C::KB; c += 128) {
+                    for (int c = sm_tid; c < nchunks * C::KB; c += 128 * C::NWG) {
                         const int kb = c / nchunks;
                         const int rem = c - kb * nchunks;
                         const int rr = rows + (rem >> 3);
@@ -403,10 +443,10 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 } else if (rows < T) {
                     bad = true;
                 }
-                uint32_t sr[RP];
+                uint32_t sr[SCOLS];
                 if (!bad && wait_bounded(&sm->s_full[j2], (i >> 1) & 1, abort_flag, budget)) {
                     tc_fence_after_sync();
-                    tmem_ld_cols<RP>(tmem + lane_addr + j2 * RP, sr);
+                    tmem_ld_cols<SCOLS>(tmem + lane_addr + j2 * RP + hbase, sr);
                     tmem_wait_ld();
                     tc_fence_before_sync();
                     __syncwarp();
@@ -414,98 +454,75 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 } else {
                     bad = true;
 #pragma unroll
-                    for (int h = 0; h < RP; ++h) sr[h] = 0u;
+                    for (int h = 0; h < SCOLS; ++h) sr[h] = 0u;
                 }
 
                 const bool valid = row < rows;
-                float x[NH];
+                float x[NHW];
 #pragma unroll
-                for (int h = 0; h < NH; ++h)
+                for (int h = 0; h < NHW; ++h)
                     x[h] = valid ? __uint_as_float(sr[h]) * p.scale_log2 : -INFINITY;
                 // Per-head maximum over the warp's 32 rows.
                 {
-                    float wm[NH];
+                    float wm[NHW];
 #pragma unroll
-                    for (int h = 0; h < NH; ++h) wm[h] = x[h];
-                    warp_max_transpose<NH, C::LOG2NH>(wm, lane);
-                    if (lane < NH)
-                        reinterpret_cast<float *>(&sm->wmax[j2][q4][0])[transpose_head<NH, C::LOG2NH>(lane)] = wm[0];
+                    for (int h = 0; h < NHW; ++h) wm[h] = x[h];
+                    warp_max_transpose<NHW, C::LOG2NHW>(wm, lane);
+                    if (lane < NHW)
+                        reinterpret_cast<float *>(&sm->wmax[wg][j2][q4][0])[transpose_head<NHW, C::LOG2NHW>(lane)] = wm[0];
                 }
-                if (named_bar_any(1, 128, bad)) {
+                if (named_bar_any(bar_id, 128, bad)) {
                     ok = false;
                     break;
                 }
-
-                if constexpr (C::REG_STATE) {
-                    // Every thread forms the tile maximum of every head from the four warp
-                    // maxima and keeps the running maximum in registers (identical in all
-                    // threads), so one barrier per tile suffices.
+                // Every thread forms the tile maximum of each of its heads from the four warp
+                // maxima and keeps the running maximum in registers (identical in all threads
+                // of the group), so one barrier per tile suffices.
 #pragma unroll
-                    for (int h4 = 0; h4 < C::NH4; ++h4) {
-                        const float4 a = sm->wmax[j2][0][h4], b = sm->wmax[j2][1][h4];
-                        const float4 c = sm->wmax[j2][2][h4], e = sm->wmax[j2][3][h4];
-                        const float t4[4] = {fmaxf(fmaxf(a.x, b.x), fmaxf(c.x, e.x)),
-                                             fmaxf(fmaxf(a.y, b.y), fmaxf(c.y, e.y)),
-                                             fmaxf(fmaxf(a.z, b.z), fmaxf(c.z, e.z)),
-                                             fmaxf(fmaxf(a.w, b.w), fmaxf(c.w, e.w))};
+                for (int h4 = 0; h4 < C::NHW4; ++h4) {
+                    const float4 a = sm->wmax[wg][j2][0][h4], b = sm->wmax[wg][j2][1][h4];
+                    const float4 c = sm->wmax[wg][j2][2][h4], e = sm->wmax[wg][j2][3][h4];
+                    const float t4[4] = {fmaxf(fmaxf(a.x, b.x), fmaxf(c.x, e.x)),
+                                         fmaxf(fmaxf(a.y, b.y), fmaxf(c.y, e.y)),
+                                         fmaxf(fmaxf(a.z, b.z), fmaxf(c.z, e.z)),
+                                         fmaxf(fmaxf(a.w, b.w), fmaxf(c.w, e.w))};
 #pragma unroll
-                        for (int e4 = 0; e4 < 4; ++e4) {
-                            const int h = h4 * 4 + e4;
-                            if (h < NH) {
-                                const float m_new = fmaxf(m_run[h], t4[e4]);
-                                alpha[h] = m_new == -INFINITY ? 0.f : ex2_approx(m_run[h] - m_new);
-                                m_run[h] = m_new;
-                            }
+                    for (int e4 = 0; e4 < 4; ++e4) {
+                        const int h = h4 * 4 + e4;
+                        if (h < NHW) {
+                            const float m_new = fmaxf(m_run[h], t4[e4]);
+                            alpha[h] = m_new == -INFINITY ? 0.f : ex2_approx(m_run[h] - m_new);
+                            m_run[h] = m_new;
                         }
                     }
-                } else {
-                    if (wg_tid < nh) {
-                        const int h = wg_tid;
-                        const float *wf = reinterpret_cast<const float *>(&sm->wmax[j2][0][0]);
-                        constexpr int WS = 4 * C::NH4;  // floats per warp row
-                        const float tmax = fmaxf(fmaxf(wf[h], wf[WS + h]), fmaxf(wf[2 * WS + h], wf[3 * WS + h]));
-                        const float m_old = jj == 0 ? -INFINITY : sm->mcur[j2 ^ 1][h];
-                        const float m_new = fmaxf(m_old, tmax);
-                        sm->mcur[j2][h] = m_new;
-                        sm->alpha[j2][h] = jj == 0 ? 0.f : ex2_approx(m_old - m_new);
-                    }
-                    named_bar_sync(1, 128);  // every thread of the group arrives here
                 }
 
                 // P = hi + lo in bf16 (~16 significant bits).  This thread's tile row is K row
-                // `row` of the MN-major P^T: high parts at values [0, RP), low parts at [RP, 2RP),
-                // written as 16-byte chunks of 8 heads.
+                // `row` of the MN-major P^T: high parts at values [0, RP), low parts at
+                // [RP, 2RP), written as 16-byte chunks of 8 heads.
                 {
                     uint8_t *prow = p_base + j2 * C::P_BYTES + row * C::P_ROWB;
                     const int swz = C::P_ROWB == 128 ? (row & 7) : ((row >> 1) & 3);
                     constexpr int HALF_VALS = C::P_ROWB / 2;  // bf16 values per atom row
 #pragma unroll
-                    for (int h = 0; h < NH; ++h) {
-                        float m_h, a_h;
-                        if constexpr (C::REG_STATE) {
-                            m_h = m_run[h];
-                            a_h = alpha[h];
-                        } else {
-                            m_h = sm->mcur[j2][h];
-                            a_h = sm->alpha[j2][h];
-                        }
-                        x[h] = ex2_approx(x[h] - m_h);  // x now holds p
-                        l[h] = l[h] * a_h + x[h];
+                    for (int h = 0; h < NHW; ++h) {
+                        x[h] = ex2_approx(x[h] - m_run[h]);  // x now holds p
+                        l[h] = l[h] * alpha[h] + x[h];
                     }
 #pragma unroll
-                    for (int c8 = 0; c8 < (NH + 7) / 8; ++c8) {
+                    for (int c8 = 0; c8 < (NHW + 7) / 8; ++c8) {
                         uint32_t hw[4], lw[4];
 #pragma unroll
                         for (int w2 = 0; w2 < 4; ++w2) {
                             const int h = c8 * 8 + 2 * w2;
-                            const float a = h < NH ? x[h] : 0.f;
-                            const float b = h + 1 < NH ? x[h + 1] : 0.f;
+                            const float a = h < NHW ? x[h] : 0.f;
+                            const float b = h + 1 < NHW ? x[h + 1] : 0.f;
                             const __nv_bfloat162 hi = __floats2bfloat162_rn(a, b);
                             const __nv_bfloat162 lo = __floats2bfloat162_rn(a - __low2float(hi), b - __high2float(hi));
                             hw[w2] = *reinterpret_cast<const uint32_t *>(&hi);
                             lw[w2] = *reinterpret_cast<const uint32_t *>(&lo);
                         }
-                        const int eh = c8 * 8, el = RP + c8 * 8;
+                        const int eh = hbase + c8 * 8, el = RP + hbase + c8 * 8;
                         *reinterpret_cast<uint4 *>(prow + (eh / HALF_VALS) * C::P_ATOMB + ((((eh % HALF_VALS) >> 3) ^ swz) << 4)) =
                             make_uint4(hw[0], hw[1], hw[2], hw[3]);
                         *reinterpret_cast<uint4 *>(prow + (el / HALF_VALS) * C::P_ATOMB + ((((el % HALF_VALS) >> 3) ^ swz) << 4)) =
@@ -525,22 +542,17 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         continue;
                     }
                     tc_fence_after_sync();
-                    const uint32_t obase = tmem + lane_addr + C::O_COL + jt * C::O_COL;
+                    const uint32_t obase = tmem + lane_addr + C::O_COL + jt * C::O_COL + hbase;
 #pragma unroll
-                    for (int c = 0; c < NH; c += 16) {
+                    for (int c = 0; c < NHW; c += 16) {
                         uint32_t hi[16], lo[16];
                         tmem_ld16(obase + c, hi);
                         tmem_ld16(obase + RP + c, lo);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            if (c + e < NH) {
-                                float a_h;
-                                if constexpr (C::REG_STATE) a_h = alpha[c + e];
-                                else a_h = sm->alpha[j2][c + e];
-                                O[c + e] = (O[c + e] + (__uint_as_float(hi[e]) + __uint_as_float(lo[e]))) * a_h;
-                            }
-                        }
+                        for (int e = 0; e < 16; ++e)
+                            if (c + e < NHW)
+                                O[c + e] = (O[c + e] + (__uint_as_float(hi[e]) + __uint_as_float(lo[e]))) * alpha[c + e];
                     }
                     tc_fence_before_sync();
                     __syncwarp();
@@ -552,16 +564,16 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 // Last tile of the piece: its O is already relative to the final max.
                 const int jt = (i - 1) & 1;
                 tc_fence_after_sync();
-                const uint32_t obase = tmem + lane_addr + C::O_COL + jt * C::O_COL;
+                const uint32_t obase = tmem + lane_addr + C::O_COL + jt * C::O_COL + hbase;
 #pragma unroll
-                for (int c = 0; c < NH; c += 16) {
+                for (int c = 0; c < NHW; c += 16) {
                     uint32_t hi[16], lo[16];
                     tmem_ld16(obase + c, hi);
                     tmem_ld16(obase + RP + c, lo);
                     tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 16; ++e)
-                        if (c + e < NH) O[c + e] += __uint_as_float(hi[e]) + __uint_as_float(lo[e]);
+                        if (c + e < NHW) O[c + e] += __uint_as_float(hi[e]) + __uint_as_float(lo[e]);
                 }
                 tc_fence_before_sync();
                 __syncwarp();
@@ -571,22 +583,22 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             // Sum of the softmax numerators over the 128 rows of every tile of the piece.
 #pragma unroll
-            for (int h = 0; h < NH; ++h) {
-                const float s = warp_sum_f32(l[h]);
-                if (lane == 0 && h < nh) sm->lsum[q4][h] = s;
+            for (int h = 0; h < NHW; ++h) {
+                const float sum = warp_sum_f32(l[h]);
+                if (lane == 0) sm->lsum[wg][q4][h] = sum;
             }
-            if (named_bar_any(1, 128, bad)) {
+            if (named_bar_any(bar_id, 128, bad)) {
                 ok = false;
                 break;
             }
             if (dcol >= 0) {
-                const int h0 = sg.kvh * p.r + sg.hb * p.RB;
+                const int h0 = sg.kvh * p.r + sg.hb * p.RB + hbase;
                 if (sg.whole) {
                     float *o = p.out + (static_cast<long long>(sg.b) * p.H_q + h0) * D + dcol;
 #pragma unroll
-                    for (int h = 0; h < NH; ++h) {
-                        if (h < nh) {
-                            const float L = sm->lsum[0][h] + sm->lsum[1][h] + sm->lsum[2][h] + sm->lsum[3][h];
+                    for (int h = 0; h < NHW; ++h) {
+                        if (h < nhw) {
+                            const float L = sm->lsum[wg][0][h] + sm->lsum[wg][1][h] + sm->lsum[wg][2][h] + sm->lsum[wg][3][h];
                             o[static_cast<long long>(h) * D] = O[h] / L;
                         }
                     }
@@ -594,25 +606,21 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     float *slot = p.ws + p.hdr_floats +
                                   (static_cast<long long>(blockIdx.x) + sg.unit) * p.slot_floats;
 #pragma unroll
-                    for (int h = 0; h < NH; ++h)
-                        if (h < nh) slot[h * D + dcol] = O[h];
-                    if (dcol < nh) {
+                    for (int h = 0; h < NHW; ++h)
+                        if (h < nhw) slot[(hbase + h) * D + dcol] = O[h];
+                    if (dcol < nhw) {
                         const int h = dcol;
                         float m_final = -INFINITY;
-                        if constexpr (C::REG_STATE) {
 #pragma unroll
-                            for (int hh = 0; hh < NH; ++hh)
-                                if (hh == h) m_final = m_run[hh];
-                        } else {
-                            m_final = sm->mcur[j2][h];
-                        }
-                        slot[nh * D + h] = m_final;
-                        slot[nh * D + nh + h] = sm->lsum[0][h] + sm->lsum[1][h] + sm->lsum[2][h] + sm->lsum[3][h];
+                        for (int hh = 0; hh < NHW; ++hh)
+                            if (hh == h) m_final = m_run[hh];
+                        slot[nh * D + hbase + h] = m_final;
+                        slot[nh * D + nh + hbase + h] = sm->lsum[wg][0][h] + sm->lsum[wg][1][h] + sm->lsum[wg][2][h] + sm->lsum[wg][3][h];
                     }
                 }
             }
             // the next piece rewrites lsum only after every thread has read it
-            named_bar_sync(1, 128);
+            named_bar_sync(bar_id, 128);
         }
         if (!ok) fail();
     }
@@ -623,10 +631,10 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (warp == 0) tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
-template <int D, int NH>
+template <int D, int NH, bool PAGED>
 static int launch_split_tc_impl(const TmaMaps &maps, const DecodeParams &p, cudaStream_t stream) {
     using C = TcCfg<D, NH>;
-    auto kern = split_tc_kernel<D, NH>;
+    auto kern = split_tc_kernel<D, NH, PAGED>;
     static bool attr_set[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return GQA_ERR_CUDA;
@@ -637,7 +645,7 @@ static int launch_split_tc_impl(const TmaMaps &maps, const DecodeParams &p, cuda
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.G);
-    cfg.blockDim = dim3(192);
+    cfg.blockDim = dim3(C::THREADS);
     cfg.dynamicSmemBytes = C::SMEM_BYTES;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -650,16 +658,16 @@ static int launch_split_tc_impl(const TmaMaps &maps, const DecodeParams &p, cuda
     return GQA_OK;
 }
 
-template <int D>
+template <int D, bool PAGED>
 static int launch_split_tc_d(const TmaMaps &maps, const DecodeParams &p, int nh, cudaStream_t stream) {
     switch (nh) {
-        case 1: return launch_split_tc_impl<D, 1>(maps, p, stream);
-        case 2: return launch_split_tc_impl<D, 2>(maps, p, stream);
-        case 4: return launch_split_tc_impl<D, 4>(maps, p, stream);
-        case 8: return launch_split_tc_impl<D, 8>(maps, p, stream);
-        case 16: return launch_split_tc_impl<D, 16>(maps, p, stream);
-        case 32: return launch_split_tc_impl<D, 32>(maps, p, stream);
-        default: return launch_split_tc_impl<D, 64>(maps, p, stream);
+        case 1: return launch_split_tc_impl<D, 1, PAGED>(maps, p, stream);
+        case 2: return launch_split_tc_impl<D, 2, PAGED>(maps, p, stream);
+        case 4: return launch_split_tc_impl<D, 4, PAGED>(maps, p, stream);
+        case 8: return launch_split_tc_impl<D, 8, PAGED>(maps, p, stream);
+        case 16: return launch_split_tc_impl<D, 16, PAGED>(maps, p, stream);
+        case 32: return launch_split_tc_impl<D, 32, PAGED>(maps, p, stream);
+        default: return launch_split_tc_impl<D, 64, PAGED>(maps, p, stream);
     }
 }
 
@@ -678,8 +686,11 @@ int tc_q_box_rows(int heads_per_unit) {
 
 int launch_split_tc(const TmaMaps &maps, const DecodeParams &p, cudaStream_t stream) {
     const int nh = tc_heads_bucket(p.RB);
-    return p.d == 128 ? launch_split_tc_d<128>(maps, p, nh, stream)
-                      : launch_split_tc_d<64>(maps, p, nh, stream);
+    if (p.block_table != nullptr)
+        return p.d == 128 ? launch_split_tc_d<128, true>(maps, p, nh, stream)
+                          : launch_split_tc_d<64, true>(maps, p, nh, stream);
+    return p.d == 128 ? launch_split_tc_d<128, false>(maps, p, nh, stream)
+                      : launch_split_tc_d<64, false>(maps, p, nh, stream);
 }
 
 }  // namespace gqa

@@ -21,6 +21,10 @@ int tc_q_box_rows(int heads_per_unit);
 int launch_split_f32(const DecodeParams &p, const float *q, const float *kc, const float *vc,
                      cudaStream_t stream);
 int launch_combine(const DecodeParams &p, cudaStream_t stream);
+int launch_append_paged(const void *k_new, const void *v_new, void *k_pool, void *v_pool,
+                        const int32_t *block_table, int max_pages, int32_t *seq_lens, int B,
+                        int H_kv, int row_bytes, int page_size, int n_pages, int32_t *status,
+                        cudaStream_t stream);
 int launch_append(const void *k_new, const void *v_new, void *k_cache, void *v_cache,
                   int32_t *seq_lens, int B, int H_kv, int row_bytes, int L_max, int32_t *status,
                   cudaStream_t stream);

@@ -32,6 +32,12 @@ struct DecodeParams {
     int UB;    // units per sequence = H_kv * HB
     int T;     // cached rows per tile
     int G;     // CTAs of the split kernel
+    int window;  // > 0: attend only the last `window` rows of each sequence; 0: all rows
+    // Paged cache (block_table != nullptr): row t of sequence b is row t % page_size of page
+    // block_table[b * max_pages + t / page_size] of a pool of n_pages pages; L_max is then
+    // max_pages * page_size.
+    const int32_t *block_table;
+    int max_pages, page_size, n_pages;
     float scale_log2;                 // softmax scale * log2(e)
     unsigned long long wait_ns;       // bound of every pipeline wait
     long long slot_floats;            // RB * (d + 2)
@@ -43,6 +49,16 @@ __device__ __forceinline__ int valid_len(int n, int L_max) {
 }
 
 __device__ __forceinline__ int tiles_of(int n, int T) { return (n + T - 1) / T; }
+
+// First attended row of a sequence with n rows: n - window under a sliding window, else 0.
+__device__ __forceinline__ int first_row(int n, int window) {
+    return (window > 0 && n > window) ? n - window : 0;
+}
+
+// Tiles of a sequence with (valid) length n.
+__device__ __forceinline__ int seq_tiles(int n, const DecodeParams &p) {
+    return tiles_of(n - first_row(n, p.window), p.T);
+}
 
 __device__ __forceinline__ long long cta_range_begin(long long i, long long total, long long G) {
     return i * total / G;
@@ -82,7 +98,7 @@ __device__ inline CtaRange locate_cta_range(const DecodeParams &p, int cta, int 
             n = valid_len(raw, p.L_max);
             if (flag_range && n != raw && p.status != nullptr) atomicOr(p.status, GQA_STATUS_SEQLEN_RANGE);
         }
-        const long long v = static_cast<long long>(tiles_of(n, p.T)) * p.UB;
+        const long long v = static_cast<long long>(seq_tiles(n, p)) * p.UB;
         const long long incl = warp_incl_scan(v, lane);
         if (hdr != nullptr && b < p.B) hdr[b] = run + incl - v;
         run += __shfl_sync(kFullMask, incl, 31);
@@ -99,7 +115,7 @@ __device__ inline CtaRange locate_cta_range(const DecodeParams &p, int cta, int 
     for (int base = 0; base < p.B; base += 32) {
         const int b = base + lane;
         const int n = b < p.B ? valid_len(p.seq_lens[b], p.L_max) : 0;
-        const long long v = static_cast<long long>(tiles_of(n, p.T)) * p.UB;
+        const long long v = static_cast<long long>(seq_tiles(n, p)) * p.UB;
         const long long incl = warp_incl_scan(v, lane);
         const long long excl = incl - v;
         const bool hit = v > 0 && off + excl <= cr.begin && cr.begin < off + incl;
@@ -119,7 +135,8 @@ __device__ inline CtaRange locate_cta_range(const DecodeParams &p, int cta, int 
 struct Segment {
     int b, kvh, hb;  // sequence, key/value head, block of query heads
     int j0, len;     // first tile (within the unit) and number of tiles of the piece
-    int n;           // rows attended by sequence b
+    int n;           // rows in sequence b
+    int first;       // first attended row (0 unless a sliding window cuts the front)
     int unit;        // unit index b * UB + (kvh * HB + hb)
     bool whole;      // the piece is the entire unit
 };
@@ -128,7 +145,7 @@ struct Segment {
 // all of them see the same sequence of segments.
 struct SegmentWalker {
     const int32_t *lens;
-    int B, UB, HB, L_max, T;
+    int B, UB, HB, L_max, T, window;
     int b, n, nt;
     long long off, t, end;
 
@@ -139,13 +156,14 @@ struct SegmentWalker {
         HB = p.HB;
         L_max = p.L_max;
         T = p.T;
+        window = p.window;
         t = cr.begin;
         end = cr.end;
         b = cr.b0;
         off = cr.off0;
         if (t < end) {
             n = valid_len(lens[b], L_max);
-            nt = tiles_of(n, T);
+            nt = tiles_of(n - first_row(n, window), T);
         } else {
             n = 0;
             nt = 0;
@@ -161,7 +179,7 @@ struct SegmentWalker {
                 return false;
             }
             n = valid_len(lens[b], L_max);
-            nt = tiles_of(n, T);
+            nt = tiles_of(n - first_row(n, window), T);
         }
         const long long rel = t - off;
         const int k = static_cast<int>(rel / nt);
@@ -174,6 +192,7 @@ struct SegmentWalker {
         s.j0 = j0;
         s.len = len;
         s.n = n;
+        s.first = first_row(n, window);
         s.unit = b * UB + k;
         s.whole = (j0 == 0 && len == nt);
         t += len;

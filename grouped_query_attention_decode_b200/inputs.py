@@ -38,6 +38,7 @@ class Workload:
     seed: int
     length: int | None = None          # fixed attended length; None = ragged U{1..L_max}
     scale: float | None = None         # None = 1/sqrt(d)
+    window: int = 0                    # > 0: sliding window, attend the last `window` rows
     note: str = field(default="", compare=False)
 
     @property
@@ -73,6 +74,9 @@ WORKLOADS = {
         Workload("ragged_long", B=32, H_q=32, H_kv=8, d=128, L_max=32768, dtype=torch.bfloat16,
                  q_std=1.0, kv_std=1.0, seed=4, length=None,
                  note="ragged long-context batch, lengths uniform in [1, 32768]"),
+        Workload("ragged_long_window4096", B=32, H_q=32, H_kv=8, d=128, L_max=32768,
+                 dtype=torch.bfloat16, q_std=1.0, kv_std=1.0, seed=4, length=None, window=4096,
+                 note="the ragged batch with a Mistral-style sliding window of 4096 rows"),
     ]
 }
 
@@ -127,6 +131,13 @@ def make_inputs(w: Workload, lengths=None, poison: bool = False) -> dict:
     }
 
 
+def attended_rows(w: Workload, n: int) -> int:
+    """Rows a sequence of length n attends: all of them, or the last `window`."""
+    n = int(n)
+    return min(n, w.window) if w.window > 0 else n
+
+
 def ideal_kv_bytes(w: Workload, lengths) -> int:
-    """K and V bytes one decode step must read: 2 * sum(n_b) * H_kv * d * element size."""
-    return 2 * int(sum(int(n) for n in lengths)) * w.H_kv * w.d * w.elem_bytes
+    """K and V bytes one decode step must read: 2 * sum(attended rows) * H_kv * d * element
+    size."""
+    return 2 * int(sum(attended_rows(w, n) for n in lengths)) * w.H_kv * w.d * w.elem_bytes

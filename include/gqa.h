@@ -75,6 +75,9 @@ typedef enum {
 #define GQA_STATUS_WAIT_TIMEOUT 4     /* gqa_decode: a pipeline wait ran past its time limit;
                                          the affected outputs are not valid */
 #define GQA_STATUS_INTERNAL 8         /* gqa_decode: shared-memory base not 1024-byte aligned */
+#define GQA_STATUS_PAGE_RANGE 16      /* paged calls: a block-table entry a row needs is outside
+                                         [0, n_pages); page 0 was read instead, the affected
+                                         outputs are not valid */
 
 /*
  * gqa_kv_append: write this step's key and value vectors into the cache.
@@ -130,6 +133,50 @@ int gqa_decode(const void *q, const void *k_cache, const void *v_cache, const in
                int B, int H_q, int H_kv, int d, int L_max, float scale, gqa_dtype_t dtype,
                float *out, void *workspace, size_t workspace_bytes, int32_t *status,
                cudaStream_t stream);
+
+/*
+ * gqa_decode_window: gqa_decode with a sliding window.  Each query head of sequence b attends
+ * only the last `window` cached rows, [max(0, n - window), n), n = seq_lens[b]; the rows before
+ * them are not read.  "GQA 阅读笔记", section on what came after GQA (the Mistral 7B paragraph:
+ * every token attends only the previous W = 4096 tokens, which bounds the cache a step reads by
+ * W instead of L); "从MHA到GQA" lists sliding-window attention among the methods that combine
+ * with GQA.  window must be >= 1 (GQA_ERR_SHAPE otherwise); window >= n is the full decode.
+ * Every other argument, layout and error is that of gqa_decode, and it uses the same
+ * workspace size.
+ */
+int gqa_decode_window(const void *q, const void *k_cache, const void *v_cache,
+                      const int32_t *seq_lens, int B, int H_q, int H_kv, int d, int L_max,
+                      int window, float scale, gqa_dtype_t dtype, float *out, void *workspace,
+                      size_t workspace_bytes, int32_t *status, cudaStream_t stream);
+
+/*
+ * Paged KV cache.  "GQA 阅读笔记", section on what came after GQA (the vLLM PagedAttention
+ * paragraph: the KV cache is managed in fixed-size blocks) and "GQA 深入理解", section 8
+ * (PagedAttention organises the cache to cut fragmentation).  All sequences share one pool
+ *     k_pool, v_pool  [n_pages][page_size][H_kv][d]
+ * and block_table [B][max_pages] (int32, device) names, for every sequence b, the page holding
+ * its rows [j*page_size, (j+1)*page_size): row t of sequence b is
+ *     k_pool[block_table[b][t / page_size]][t % page_size].
+ * Only the entries covering rows < seq_lens[b] (after the append: < seq_lens[b] + 1) are read.
+ * page_size must be a multiple of 8 and, for bf16, divide 128 or be a multiple of 128.  A
+ * sequence's capacity is max_pages * page_size rows (the L_max of the contiguous calls).
+ *
+ * gqa_kv_append_paged: the append of gqa_kv_append into the pool: row t = seq_lens[b] goes to
+ * page block_table[b][t / page_size], row t % page_size; then seq_lens[b] = t + 1.  A full
+ * sequence, or a page index outside [0, n_pages), is skipped with GQA_STATUS_APPEND_OVERFLOW.
+ *
+ * gqa_decode_paged: gqa_decode over the paged cache; same q, out, scale, workspace (the same
+ * gqa_decode_workspace_size) and errors.  An out-of-range page index sets GQA_STATUS_PAGE_RANGE.
+ */
+int gqa_kv_append_paged(const void *k_new, const void *v_new, void *k_pool, void *v_pool,
+                        const int32_t *block_table, int max_pages, int32_t *seq_lens, int B,
+                        int H_kv, int d, int page_size, int n_pages, gqa_dtype_t dtype,
+                        int32_t *status, cudaStream_t stream);
+int gqa_decode_paged(const void *q, const void *k_pool, const void *v_pool,
+                     const int32_t *block_table, int max_pages, const int32_t *seq_lens, int B,
+                     int H_q, int H_kv, int d, int page_size, int n_pages, float scale,
+                     gqa_dtype_t dtype, float *out, void *workspace, size_t workspace_bytes,
+                     int32_t *status, cudaStream_t stream);
 
 /*
  * gqa_decode_noalloc: gqa_decode without a caller-provided workspace.  (The pages have no

@@ -57,6 +57,15 @@ class Oracle:
         self.lib.oracle_gqa_decode.argtypes = [dp, dp, dp, ip, c_int, c_int, c_int, c_int, c_int,
                                                ctypes.c_double, dp, c_int, ip]
         self.lib.oracle_gqa_decode.restype = c_int
+        self.lib.oracle_gqa_decode_window.argtypes = [dp, dp, dp, ip, c_int, c_int, c_int, c_int,
+                                                      c_int, c_int, ctypes.c_double, dp, c_int, ip]
+        self.lib.oracle_gqa_decode_window.restype = c_int
+        self.lib.oracle_paged_gather.argtypes = [dp, ip, ip, c_int, c_int, c_int, c_int, c_int,
+                                                 c_int, dp, ip]
+        self.lib.oracle_paged_gather.restype = None
+        self.lib.oracle_kv_append_paged.argtypes = [dp, dp, dp, dp, ip, ip, c_int, c_int, c_int,
+                                                    c_int, c_int, c_int, ip]
+        self.lib.oracle_kv_append_paged.restype = None
         self.lib.oracle_max_threads.argtypes = []
         self.lib.oracle_max_threads.restype = c_int
 
@@ -122,6 +131,61 @@ class Oracle:
         if rc != 0:
             raise ValueError("oracle_gqa_decode rejected the shapes (H_q % H_kv != 0?)")
         return (out, int(status[0])) if return_status else out
+
+
+    def decode_window(self, q, k_cache, v_cache, seq_lens, window: int, scale: float,
+                      nthreads: int = 0):
+        """Like decode, but each sequence attends only its last `window` rows (window <= 0:
+        all rows)."""
+        q, kc, vc = self._f64(q), self._f64(k_cache), self._f64(v_cache)
+        lens = np.ascontiguousarray(seq_lens, dtype=np.int32)
+        B, H_q, d = q.shape
+        _, L_max, H_kv, _ = kc.shape
+        out = np.zeros((B, H_q, d), dtype=np.float64)
+        status = np.zeros(1, dtype=np.int32)
+        rc = self.lib.oracle_gqa_decode_window(self._dp(q), self._dp(kc), self._dp(vc),
+                                               self._ip(lens), B, H_q, H_kv, d, L_max, int(window),
+                                               float(scale), self._dp(out), int(nthreads),
+                                               self._ip(status))
+        if rc != 0:
+            raise ValueError("oracle_gqa_decode_window rejected the shapes")
+        return out
+
+
+    def paged_gather(self, pool, block_table, seq_lens):
+        """Logical caches [B, max_pages*page_size, H_kv, d] of a paged pool
+        [n_pages, page_size, H_kv, d]; rows >= seq_lens[b] are zero.  Returns (cache, status)."""
+        pool = self._f64(pool)
+        bt = np.ascontiguousarray(block_table, dtype=np.int32)
+        lens = np.ascontiguousarray(seq_lens, dtype=np.int32)
+        n_pages, P, H_kv, d = pool.shape
+        B, max_pages = bt.shape
+        cache = np.zeros((B, max_pages * P, H_kv, d), dtype=np.float64)
+        status = np.zeros(1, dtype=np.int32)
+        self.lib.oracle_paged_gather(self._dp(pool), self._ip(bt), self._ip(lens), B, max_pages, P,
+                                     n_pages, H_kv, d, self._dp(cache), self._ip(status))
+        return cache, int(status[0])
+
+    def kv_append_paged(self, k_new, v_new, k_pool, v_pool, block_table, seq_lens):
+        """Paged append (in place on the float64 pools and int32 lengths).  Returns status."""
+        assert k_pool.dtype == np.float64 and k_pool.flags.c_contiguous
+        assert v_pool.dtype == np.float64 and v_pool.flags.c_contiguous
+        assert seq_lens.dtype == np.int32 and seq_lens.flags.c_contiguous
+        bt = np.ascontiguousarray(block_table, dtype=np.int32)
+        n_pages, P, H_kv, d = k_pool.shape
+        B, max_pages = bt.shape
+        kn, vn = self._f64(k_new), self._f64(v_new)
+        status = np.zeros(1, dtype=np.int32)
+        self.lib.oracle_kv_append_paged(self._dp(kn), self._dp(vn), self._dp(k_pool), self._dp(v_pool),
+                                        self._ip(bt), self._ip(seq_lens), B, max_pages, P, n_pages,
+                                        H_kv, d, self._ip(status))
+        return int(status[0])
+
+    def decode_paged(self, q, k_pool, v_pool, block_table, seq_lens, scale: float):
+        """The paged decode: gather each sequence's rows from the pool, then decode."""
+        kc, st1 = self.paged_gather(k_pool, block_table, seq_lens)
+        vc, st2 = self.paged_gather(v_pool, block_table, seq_lens)
+        return self.decode(q, kc, vc, seq_lens, scale)
 
 
 _default: Oracle | None = None

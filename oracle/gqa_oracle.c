@@ -112,16 +112,23 @@ void oracle_attend_one_head(const double *q, const double *K, const double *V, i
     free(s);
 }
 
-/* One decode step's attention for every sequence and query head.
+/* One decode step's attention for every sequence and query head, optionally restricted to a
+ * sliding window.
  *   q       [B][H_q][d]
  *   k_cache [B][L_max][H_kv][d], v_cache alike
  *   seq_lens[B]: rows each sequence attends over (already counting this step's appended row)
+ *   window  > 0: every query head of sequence b attends only the last `window` rows,
+ *           [max(0, n - window), n) ("GQA 阅读笔记", section on what came after GQA, Mistral
+ *           7B paragraph: each token attends only the previous W tokens); <= 0: all n rows
  *   out     [B][H_q][d]
+ * Per sequence: expand the attended rows (re-based so the window's first row is row 0), then
+ * run textbook attention per query head.
  * Returns 0, or -1 when H_q is not a multiple of H_kv (the lesson page "r-tf2-gqa" requires
  * h to be divisible by g) or a size is not positive.  nthreads <= 0 uses the OpenMP default. */
-int oracle_gqa_decode(const double *q, const double *k_cache, const double *v_cache,
-                      const int32_t *seq_lens, int B, int H_q, int H_kv, int d, int L_max,
-                      double scale, double *out, int nthreads, int32_t *status) {
+int oracle_gqa_decode_window(const double *q, const double *k_cache, const double *v_cache,
+                             const int32_t *seq_lens, int B, int H_q, int H_kv, int d, int L_max,
+                             int window, double scale, double *out, int nthreads,
+                             int32_t *status) {
     if (B < 0 || H_q <= 0 || H_kv <= 0 || d <= 0 || L_max < 0 || H_q % H_kv != 0) return -1;
 #ifdef _OPENMP
     if (nthreads > 0) omp_set_num_threads(nthreads);
@@ -134,22 +141,93 @@ int oracle_gqa_decode(const double *q, const double *k_cache, const double *v_ca
             if (status) *status |= ORACLE_SEQLEN_RANGE;
             n = 0;
         }
+        int first = (window > 0 && n > window) ? n - window : 0;
+        int span = n - first;
         size_t per_seq = (size_t)L_max * H_kv * d;
-        size_t expanded = (size_t)n * H_q * d;
+        size_t row0 = (size_t)first * H_kv * d;
+        size_t expanded = (size_t)span * H_q * d;
         double *Kx = (double *)malloc(sizeof(double) * (expanded ? expanded : 1));
         double *Vx = (double *)malloc(sizeof(double) * (expanded ? expanded : 1));
-        oracle_expand_kv(k_cache + (size_t)b * per_seq, n, H_q, H_kv, d, Kx);
-        oracle_expand_kv(v_cache + (size_t)b * per_seq, n, H_q, H_kv, d, Vx);
+        oracle_expand_kv(k_cache + (size_t)b * per_seq + row0, span, H_q, H_kv, d, Kx);
+        oracle_expand_kv(v_cache + (size_t)b * per_seq + row0, span, H_q, H_kv, d, Vx);
 #pragma omp parallel for schedule(static)
         for (int h = 0; h < H_q; ++h) {
             oracle_attend_one_head(q + ((size_t)b * H_q + h) * d, Kx + (size_t)h * d,
-                                   Vx + (size_t)h * d, n, d, (size_t)H_q * d, scale,
+                                   Vx + (size_t)h * d, span, d, (size_t)H_q * d, scale,
                                    out + ((size_t)b * H_q + h) * d, NULL);
         }
         free(Kx);
         free(Vx);
     }
     return 0;
+}
+
+/* The full decode step (no window). */
+int oracle_gqa_decode(const double *q, const double *k_cache, const double *v_cache,
+                      const int32_t *seq_lens, int B, int H_q, int H_kv, int d, int L_max,
+                      double scale, double *out, int nthreads, int32_t *status) {
+    return oracle_gqa_decode_window(q, k_cache, v_cache, seq_lens, B, H_q, H_kv, d, L_max, 0,
+                                    scale, out, nthreads, status);
+}
+
+/* Paged KV cache ("GQA 阅读笔记", what came after GQA, the vLLM PagedAttention paragraph: the
+ * cache is managed in fixed-size blocks; "GQA 深入理解", section 8: PagedAttention organises
+ * the cache to cut fragmentation).  The cache of all sequences is one pool of pages
+ *   pool [n_pages][page_size][H_kv][d]
+ * and block_table[b][j] names the page that holds rows [j*page_size, (j+1)*page_size) of
+ * sequence b.  Row t of sequence b is pool[block_table[b][t / page_size]][t % page_size].
+ *
+ * oracle_paged_gather writes the logical cache [B][max_pages*page_size][H_kv][d] of every
+ * sequence (rows >= seq_lens[b] are left untouched); the paged decode is oracle_gqa_decode on
+ * that gathered cache.  A page index outside [0, n_pages) for a row below seq_lens[b] sets
+ * bit 4 of *status and that row is left untouched. */
+void oracle_paged_gather(const double *pool, const int32_t *block_table, const int32_t *seq_lens,
+                         int B, int max_pages, int page_size, int n_pages, int H_kv, int d,
+                         double *cache, int32_t *status) {
+    size_t L = (size_t)max_pages * page_size;
+    size_t row = (size_t)H_kv * d;
+    for (int b = 0; b < B; ++b) {
+        int n = seq_lens[b];
+        if (n < 0 || (size_t)n > L) n = 0;
+        for (int t = 0; t < n; ++t) {
+            int page = block_table[(size_t)b * max_pages + t / page_size];
+            if (page < 0 || page >= n_pages) {
+                if (status) *status |= 4;
+                continue;
+            }
+            const double *src = pool + ((size_t)page * page_size + t % page_size) * row;
+            double *dst = cache + ((size_t)b * L + t) * row;
+            for (size_t i = 0; i < row; ++i) dst[i] = src[i];
+        }
+    }
+}
+
+/* The append of a paged cache: row t = seq_lens[b] goes to page block_table[b][t / page_size]
+ * at row t % page_size; the length grows by one.  A full sequence (t >= max_pages*page_size)
+ * or a page index outside [0, n_pages) is refused with bit 1 of *status. */
+void oracle_kv_append_paged(const double *k_new, const double *v_new, double *k_pool,
+                            double *v_pool, const int32_t *block_table, int32_t *seq_lens, int B,
+                            int max_pages, int page_size, int n_pages, int H_kv, int d,
+                            int32_t *status) {
+    size_t row = (size_t)H_kv * d;
+    for (int b = 0; b < B; ++b) {
+        int t = seq_lens[b];
+        if (t < 0 || t >= max_pages * page_size) {
+            if (status) *status |= ORACLE_APPEND_OVERFLOW;
+            continue;
+        }
+        int page = block_table[(size_t)b * max_pages + t / page_size];
+        if (page < 0 || page >= n_pages) {
+            if (status) *status |= ORACLE_APPEND_OVERFLOW;
+            continue;
+        }
+        size_t dst = ((size_t)page * page_size + t % page_size) * row;
+        for (size_t i = 0; i < row; ++i) {
+            k_pool[dst + i] = k_new[(size_t)b * row + i];
+            v_pool[dst + i] = v_new[(size_t)b * row + i];
+        }
+        seq_lens[b] = t + 1;
+    }
 }
 
 /* Number of threads the OpenMP runtime will use for the next parallel region. */

@@ -272,11 +272,90 @@ def pin_divisibility(o):
     raise AssertionError("H_q % H_kv != 0 must be rejected")
 
 
+def pin_window(o):
+    """Sliding window (reading notes, what came after GQA: Mistral's W): a window at least as long
+    as the sequence is the full decode; a window of one row returns the newest V row exactly;
+    any window equals the full decode of the cache cut to its last `window` rows; and torch SDPA
+    on those rows agrees."""
+    q, K, V, lens = _rand_case(91, 3, 8, 2, 16, 40, [40, 7, 25])
+    full = o.decode(q, K, V, lens, 0.3)
+    assert np.array_equal(o.decode_window(q, K, V, lens, 40, 0.3), full)
+    assert np.array_equal(o.decode_window(q, K, V, lens, 0, 0.3), full)
+    one = o.decode_window(q, K, V, lens, 1, 0.3)
+    for b in range(3):
+        for h in range(8):
+            assert np.array_equal(one[b, h], V[b, lens[b] - 1, h // 4])
+    for W in (5, 10):
+        got = o.decode_window(q, K, V, lens, W, 0.3)
+        for b in range(3):
+            n = lens[b]
+            first = max(0, n - W)
+            cut_k = np.ascontiguousarray(K[b:b + 1, first:n])
+            cut_v = np.ascontiguousarray(V[b:b + 1, first:n])
+            want = o.decode(q[b:b + 1], cut_k, cut_v, np.array([n - first], dtype=np.int32), 0.3)
+            assert np.array_equal(got[b], want[0])
+            sd = _sdpa_reference(q[b:b + 1], cut_k, cut_v, [n - first], 0.3)
+            assert np.max(np.abs(got[b] - sd[0])) <= 1e-12
+
+
+def pin_paged(o):
+    """Paged cache (reading notes, what came after GQA: vLLM's block-managed cache): the gather
+    agrees with numpy fancy indexing; an identity block table reproduces the contiguous cache;
+    permuting the pages (with the table permuted alike) changes nothing, bit for bit; the paged
+    append lands where the contiguous append does; a missing page is refused."""
+    r = _rng(101)
+    B, P, max_pages, H_kv, d = 3, 8, 5, 2, 16
+    L = P * max_pages
+    n_pages = B * max_pages
+    lens = np.array([39, 1, 17], dtype=np.int32)
+    Kc = r.standard_normal((B, L, H_kv, d))
+    Vc = r.standard_normal((B, L, H_kv, d))
+    ident = np.arange(n_pages, dtype=np.int32).reshape(B, max_pages)
+    kpool = Kc.reshape(n_pages, P, H_kv, d).copy()
+    vpool = Vc.reshape(n_pages, P, H_kv, d).copy()
+    g, st = o.paged_gather(kpool, ident, lens)
+    assert st == 0
+    for b in range(B):
+        assert np.array_equal(g[b, :lens[b]], Kc[b, :lens[b]])
+        t = np.arange(lens[b])
+        assert np.array_equal(g[b, :lens[b]], kpool[ident[b, t // P], t % P])
+    q = r.standard_normal((B, 8, d))
+    base = o.decode(q, Kc, Vc, lens, 0.25)
+    assert np.array_equal(o.decode_paged(q, kpool, vpool, ident, lens, 0.25), base)
+    perm = r.permutation(n_pages).astype(np.int32)
+    kpool2 = np.empty_like(kpool)
+    vpool2 = np.empty_like(vpool)
+    kpool2[perm] = kpool
+    vpool2[perm] = vpool
+    table2 = perm[ident]
+    assert np.array_equal(o.decode_paged(q, kpool2, vpool2, table2, lens, 0.25), base)
+    kn = r.standard_normal((B, H_kv, d))
+    vn = r.standard_normal((B, H_kv, d))
+    l1 = lens.copy()
+    l2 = lens.copy()
+    Kc2, Vc2 = Kc.copy(), Vc.copy()
+    assert o.kv_append(kn, vn, Kc2, Vc2, l1) == 0
+    assert o.kv_append_paged(kn, vn, kpool2, vpool2, table2, l2) == 0
+    assert np.array_equal(l1, l2)
+    g2, _ = o.paged_gather(kpool2, table2, l2)
+    for b in range(B):
+        assert np.array_equal(g2[b, :l2[b]], Kc2[b, :l1[b]])
+    bad = table2.copy()
+    bad[1, l2[1] // P] = n_pages  # the page the next row of sequence 1 would go to does not exist
+    l3 = l2.copy()
+    assert o.kv_append_paged(kn, vn, kpool2, vpool2, bad, l3) & 1
+    assert l3[1] == l2[1]
+    full = l2.copy()
+    full[2] = L  # a full sequence is refused too
+    assert o.kv_append_paged(kn, vn, kpool2, vpool2, table2, full) & 1 and full[2] == L
+
+
 ALL_PINS = [
     pin_append_position, pin_append_overflow, pin_expand_matches_repeat_interleave,
     pin_single_head_vs_sdpa, pin_decode_vs_sdpa_gqa, pin_mha_endpoint, pin_mqa_endpoint,
     pin_expand_then_attend_equivalence, pin_grouping_changes_output, pin_closed_forms,
-    pin_invariants, pin_brute_force_tiny, pin_empty_and_range, pin_divisibility,
+    pin_invariants, pin_brute_force_tiny, pin_empty_and_range, pin_divisibility, pin_window,
+    pin_paged,
 ]
 
 

@@ -17,7 +17,8 @@ SRC = os.path.join(os.path.dirname(oracle_mod.__file__), "gqa_oracle.c")
 MUTANTS = {
     "group_map_modulo": ("int g = h / r;", "int g = h % H_kv;"),
     "dropped_scale": ("s[t] = scale * acc;", "s[t] = acc;"),
-    "skips_appended_row": ("int n = seq_lens[b];", "int n = seq_lens[b] - 1;"),
+    "skips_appended_row": ("int n = seq_lens[b];\n        if (n < 0 || n > L_max) {",
+                           "int n = seq_lens[b] - 1;\n        if (n < 0 || n > L_max) {"),
     "unnormalised": ("double w = s[t] / z;", "double w = s[t];"),
     "weights_keys_not_values": ("out[i] += w * V[(size_t)t * row_stride + i];",
                                 "out[i] += w * K[(size_t)t * row_stride + i];"),
@@ -27,10 +28,19 @@ MUTANTS = {
     "no_max": ("if (s[t] > m) m = s[t];", "(void)0;"),
     "append_off_by_one": ("size_t dst = (((size_t)b * L_max + t) * H_kv + g) * d + i;",
                           "size_t dst = (((size_t)b * L_max + (t ? t - 1 : 0)) * H_kv + g) * d + i;"),
-    "append_no_length_update": ("seq_lens[b] = t + 1;", "seq_lens[b] = t;"),
+    "append_no_length_update": ("v_cache[dst] = v_new[src];\n            }\n        }\n        seq_lens[b] = t + 1;",
+                                "v_cache[dst] = v_new[src];\n            }\n        }\n        seq_lens[b] = t;"),
+    "paged_append_no_length_update": ("v_pool[dst + i] = v_new[(size_t)b * row + i];\n        }\n        seq_lens[b] = t + 1;",
+                                      "v_pool[dst + i] = v_new[(size_t)b * row + i];\n        }\n        seq_lens[b] = t;"),
     "expand_wrong_head": ("out[((size_t)t * H_q + h) * d + i] = cache_b[((size_t)t * H_kv + g) * d + i];",
                           "out[((size_t)t * H_q + h) * d + i] = cache_b[((size_t)t * H_kv + (H_kv - 1 - g)) * d + i];"),
     "no_divisibility_check": ("H_q % H_kv != 0) return -1;", "0) return -1;"),
+    "paged_wrong_offset": ("const double *src = pool + ((size_t)page * page_size + t % page_size) * row;",
+                           "const double *src = pool + ((size_t)page * page_size + t / page_size) * row;"),
+    "paged_append_wrong_page": ("int page = block_table[(size_t)b * max_pages + t / page_size];\n        if (page < 0 || page >= n_pages) {\n            if (status) *status |= ORACLE_APPEND_OVERFLOW;",
+                                "int page = block_table[(size_t)b * max_pages + t % page_size];\n        if (page < 0 || page >= n_pages) {\n            if (status) *status |= ORACLE_APPEND_OVERFLOW;"),
+    "window_off_by_one": ("int first = (window > 0 && n > window) ? n - window : 0;",
+                          "int first = (window > 0 && n > window) ? n - window + 1 : 0;"),
 }
 
 
