@@ -173,7 +173,13 @@ def bench_ours(args, rank, world, local):
     assert W >= 3
     q = x["q"].to(dev)
     kn, vn = x["k_new"].to(dev), x["v_new"].to(dev)
-    caches = [(x["k_cache"].to(dev), x["v_cache"].to(dev))]
+    block_table = None
+    if w.page_size > 0:
+        paged = inputs.make_paged(x, w.page_size)
+        block_table = paged["block_table"].to(dev)
+        caches = [(paged["k_pool"].to(dev), paged["v_pool"].to(dev))]
+    else:
+        caches = [(x["k_cache"].to(dev), x["v_cache"].to(dev))]
     caches.append((caches[0][0].clone(), caches[0][1].clone()))
     lens0 = x["seq_lens_pre"].to(dev)
     out = torch.empty((w.B, w.H_q, w.d), dtype=torch.float32, device=dev)
@@ -182,6 +188,11 @@ def bench_ours(args, rank, world, local):
 
     def step(i, lens_row, qq=q, kk=kn, vv=vn):
         kc, vc = caches[i & 1]
+        if block_table is not None:
+            gqa.kv_append_paged(kk, vv, kc, vc, block_table, lens_row, status=status)
+            gqa.decode_paged(qq, kc, vc, block_table, lens_row, x["scale"], out=out, workspace=ws,
+                             status=status)
+            return
         gqa.kv_append(kk, vv, kc, vc, lens_row, status=status)
         if w.window > 0:
             gqa.decode_window(qq, kc, vc, lens_row, w.window, x["scale"], out=out, workspace=ws,
@@ -317,11 +328,12 @@ def bench_ours(args, rank, world, local):
                 "workload": w.name, "B": w.B, "H_q": w.H_q, "H_kv": w.H_kv, "d": w.d,
                 "L_max": w.L_max, "seq_len": lengths[0] if w.length else "ragged",
                 "window": w.window or None,
+                "page_size": w.page_size or None,
                 "sum_seq_lens": int(sum(lengths)), "kv_dtype": str(w.dtype).replace("torch.", ""),
                 "accumulate": "f32", "ideal_kv_bytes_per_step": ideal,
                 "parallelism": f"replicas x{world}",
                 "l2": "inputs larger than L2: two cache copies alternate between steps "
-                      f"({2 * 2 * w.B * w.L_max * w.H_kv * w.d * w.elem_bytes / 1e6:.0f} MB)",
+                      f"({2 * caches[0][0].numel() * 2 * w.elem_bytes / 1e6:.0f} MB)",
             },
             "gpu_launches": 3 * K,
             "roofline": {
@@ -397,11 +409,21 @@ def profile_run(args, local):
     x = inputs.make_inputs(w)
     q, kn, vn = x["q"].to(dev), x["k_new"].to(dev), x["v_new"].to(dev)
     kc, vc = x["k_cache"].to(dev), x["v_cache"].to(dev)
+    block_table = None
+    if w.page_size > 0:
+        paged = inputs.make_paged(x, w.page_size)
+        kc, vc = paged["k_pool"].to(dev), paged["v_pool"].to(dev)
+        block_table = paged["block_table"].to(dev)
     lens_rows = x["seq_lens_pre"].to(dev).repeat(args.warmup + args.steps, 1).contiguous()
     out = torch.empty((w.B, w.H_q, w.d), dtype=torch.float32, device=dev)
     ws = gqa.alloc_workspace(w.B, w.H_q, w.H_kv, w.d, w.dtype, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     for i in range(args.warmup + args.steps):
+        if block_table is not None:
+            gqa.kv_append_paged(kn, vn, kc, vc, block_table, lens_rows[i], status=status)
+            gqa.decode_paged(q, kc, vc, block_table, lens_rows[i], x["scale"], out=out,
+                             workspace=ws, status=status)
+            continue
         gqa.kv_append(kn, vn, kc, vc, lens_rows[i], status=status)
         if w.window > 0:
             gqa.decode_window(q, kc, vc, lens_rows[i], w.window, x["scale"], out=out,

@@ -39,6 +39,7 @@ class Workload:
     length: int | None = None          # fixed attended length; None = ragged U{1..L_max}
     scale: float | None = None         # None = 1/sqrt(d)
     window: int = 0                    # > 0: sliding window, attend the last `window` rows
+    page_size: int = 0                 # > 0: the cache lives in a paged pool (see make_paged)
     note: str = field(default="", compare=False)
 
     @property
@@ -74,6 +75,9 @@ WORKLOADS = {
         Workload("ragged_long", B=32, H_q=32, H_kv=8, d=128, L_max=32768, dtype=torch.bfloat16,
                  q_std=1.0, kv_std=1.0, seed=4, length=None,
                  note="ragged long-context batch, lengths uniform in [1, 32768]"),
+        Workload("llama2_70b_layer_paged16", B=16, H_q=64, H_kv=8, d=128, L_max=4096,
+                 dtype=torch.bfloat16, q_std=0.5, kv_std=0.5, seed=1, length=4096, page_size=16,
+                 note="the Llama-2-70B-shaped layer in a paged pool of 16-row pages"),
         Workload("ragged_long_window4096", B=32, H_q=32, H_kv=8, d=128, L_max=32768,
                  dtype=torch.bfloat16, q_std=1.0, kv_std=1.0, seed=4, length=None, window=4096,
                  note="the ragged batch with a Mistral-style sliding window of 4096 rows"),
@@ -82,9 +86,10 @@ WORKLOADS = {
 
 
 def custom(name="custom", *, B, H_q, H_kv, d, L_max, dtype=torch.bfloat16, q_std=1.0,
-           kv_std=1.0, seed=1234, length=None, scale=None) -> Workload:
+           kv_std=1.0, seed=1234, length=None, scale=None, window=0, page_size=0) -> Workload:
     return Workload(name, B=B, H_q=H_q, H_kv=H_kv, d=d, L_max=L_max, dtype=dtype, q_std=q_std,
-                    kv_std=kv_std, seed=seed, length=length, scale=scale)
+                    kv_std=kv_std, seed=seed, length=length, scale=scale, window=window,
+                    page_size=page_size)
 
 
 def _normal(shape, gen, std, dtype):
@@ -129,6 +134,26 @@ def make_inputs(w: Workload, lengths=None, poison: bool = False) -> dict:
         "q": q, "k_cache": k_cache, "v_cache": v_cache, "k_new": k_new, "v_new": v_new,
         "seq_lens_pre": seq_lens_pre, "lengths": drawn, "scale": w.softmax_scale,
     }
+
+
+def make_paged(x: dict, page_size: int, extra_pages: int = 3, seed: int = 99) -> dict:
+    """Scatter the contiguous caches of ``x`` ([B, L_max, H_kv, d], L_max a multiple of
+    page_size) into a pool of pages in a seeded random order: block_table[b, j] is the pool
+    page holding rows [j*page_size, (j+1)*page_size) of sequence b.  ``extra_pages`` unused
+    pages (NaN) are mixed in.  Returns {"k_pool", "v_pool", "block_table"}."""
+    kc, vc = x["k_cache"], x["v_cache"]
+    B, L_max, H_kv, d = kc.shape
+    assert L_max % page_size == 0
+    max_pages = L_max // page_size
+    n_pages = B * max_pages + extra_pages
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    perm = torch.randperm(n_pages, generator=g)[: B * max_pages].to(torch.int32)
+    k_pool = torch.full((n_pages, page_size, H_kv, d), float("nan"), dtype=kc.dtype)
+    v_pool = torch.full_like(k_pool, float("nan"))
+    k_pool[perm.long()] = kc.reshape(B * max_pages, page_size, H_kv, d)
+    v_pool[perm.long()] = vc.reshape(B * max_pages, page_size, H_kv, d)
+    return {"k_pool": k_pool, "v_pool": v_pool, "block_table": perm.reshape(B, max_pages).contiguous()}
 
 
 def attended_rows(w: Workload, n: int) -> int:

@@ -66,6 +66,9 @@ class Oracle:
         self.lib.oracle_kv_append_paged.argtypes = [dp, dp, dp, dp, ip, ip, c_int, c_int, c_int,
                                                     c_int, c_int, c_int, ip]
         self.lib.oracle_kv_append_paged.restype = None
+        self.lib.oracle_gqa_decode_multi.argtypes = [dp, dp, dp, ip, c_int, c_int, c_int, c_int,
+                                                     c_int, c_int, ctypes.c_double, dp, c_int, ip]
+        self.lib.oracle_gqa_decode_multi.restype = c_int
         self.lib.oracle_max_threads.argtypes = []
         self.lib.oracle_max_threads.restype = c_int
 
@@ -151,6 +154,23 @@ class Oracle:
             raise ValueError("oracle_gqa_decode_window rejected the shapes")
         return out
 
+
+    def decode_multi(self, q, k_cache, v_cache, seq_lens, scale: float, nthreads: int = 0,
+                     return_status: bool = False):
+        """Q query tokens per sequence (q [B, Q, H_q, d]); query j attends rows
+        [0, n - Q + 1 + j).  Returns out [B, Q, H_q, d]."""
+        q, kc, vc = self._f64(q), self._f64(k_cache), self._f64(v_cache)
+        lens = np.ascontiguousarray(seq_lens, dtype=np.int32)
+        B, Q, H_q, d = q.shape
+        _, L_max, H_kv, _ = kc.shape
+        out = np.zeros((B, Q, H_q, d), dtype=np.float64)
+        status = np.zeros(1, dtype=np.int32)
+        rc = self.lib.oracle_gqa_decode_multi(self._dp(q), self._dp(kc), self._dp(vc), self._ip(lens),
+                                              B, Q, H_q, H_kv, d, L_max, float(scale), self._dp(out),
+                                              int(nthreads), self._ip(status))
+        if rc != 0:
+            raise ValueError("oracle_gqa_decode_multi rejected the shapes")
+        return (out, int(status[0])) if return_status else out
 
     def paged_gather(self, pool, block_table, seq_lens):
         """Logical caches [B, max_pages*page_size, H_kv, d] of a paged pool

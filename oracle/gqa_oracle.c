@@ -170,6 +170,51 @@ int oracle_gqa_decode(const double *q, const double *k_cache, const double *v_ca
                                     scale, out, nthreads, status);
 }
 
+/* Several query tokens per sequence in one step (speculative decoding: "GQA 阅读笔记", what came
+ * after GQA and the engineering notes -- the target model checks k drafted tokens in one pass,
+ * all k queries attend the cache, which is read once).  The Q new tokens are the last Q rows
+ * of the cache, and query j (0 <= j < Q) attends rows [0, n - Q + 1 + j): the prefix plus the
+ * drafted tokens up to and including its own (causal among the drafts).
+ *   q   [B][Q][H_q][d], caches as oracle_gqa_decode, seq_lens[b] = n (>= Q), out [B][Q][H_q][d]
+ * A sequence with n < Q, n < 0 or n > L_max gets zeros and sets bit 2 of *status. */
+int oracle_gqa_decode_multi(const double *q, const double *k_cache, const double *v_cache,
+                            const int32_t *seq_lens, int B, int Q, int H_q, int H_kv, int d,
+                            int L_max, double scale, double *out, int nthreads, int32_t *status) {
+    if (B < 0 || Q <= 0 || H_q <= 0 || H_kv <= 0 || d <= 0 || L_max < 0 || H_q % H_kv != 0)
+        return -1;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+    for (int b = 0; b < B; ++b) {
+        int n = seq_lens[b];
+        if (n < Q || n > L_max) {
+            if (status) *status |= ORACLE_SEQLEN_RANGE;
+            for (size_t i = 0; i < (size_t)Q * H_q * d; ++i) out[(size_t)b * Q * H_q * d + i] = 0.0;
+            continue;
+        }
+        size_t per_seq = (size_t)L_max * H_kv * d;
+        size_t expanded = (size_t)n * H_q * d;
+        double *Kx = (double *)malloc(sizeof(double) * expanded);
+        double *Vx = (double *)malloc(sizeof(double) * expanded);
+        oracle_expand_kv(k_cache + (size_t)b * per_seq, n, H_q, H_kv, d, Kx);
+        oracle_expand_kv(v_cache + (size_t)b * per_seq, n, H_q, H_kv, d, Vx);
+        for (int j = 0; j < Q; ++j) {
+            int rows = n - Q + 1 + j;
+#pragma omp parallel for schedule(static)
+            for (int h = 0; h < H_q; ++h) {
+                size_t qi = (((size_t)b * Q + j) * H_q + h) * d;
+                oracle_attend_one_head(q + qi, Kx + (size_t)h * d, Vx + (size_t)h * d, rows, d,
+                                       (size_t)H_q * d, scale, out + qi, NULL);
+            }
+        }
+        free(Kx);
+        free(Vx);
+    }
+    return 0;
+}
+
 /* Paged KV cache ("GQA 阅读笔记", what came after GQA, the vLLM PagedAttention paragraph: the
  * cache is managed in fixed-size blocks; "GQA 深入理解", section 8: PagedAttention organises
  * the cache to cut fragmentation).  The cache of all sequences is one pool of pages

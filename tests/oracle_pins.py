@@ -350,12 +350,40 @@ def pin_paged(o):
     assert o.kv_append_paged(kn, vn, kpool2, vpool2, table2, full) & 1 and full[2] == L
 
 
+def pin_multi_query(o):
+    """Q query tokens per sequence (speculative verification): Q = 1 is the ordinary decode;
+    query j equals the ordinary decode of the cache cut to its first n - Q + 1 + j rows; and
+    torch SDPA with the bottom-right-aligned causal mask agrees."""
+    r = _rng(111)
+    B, Q, H_q, H_kv, d, L = 3, 4, 8, 2, 16, 30
+    lens = np.array([30, 4, 17], dtype=np.int32)
+    q = r.standard_normal((B, Q, H_q, d))
+    K = r.standard_normal((B, L, H_kv, d))
+    V = r.standard_normal((B, L, H_kv, d))
+    one = o.decode_multi(q[:, :1], K, V, lens, 0.3)
+    assert np.array_equal(one[:, 0], o.decode(q[:, 0], K, V, lens, 0.3))
+    got = o.decode_multi(q, K, V, lens, 0.3)
+    for j in range(Q):
+        cut = lens - Q + 1 + j
+        assert np.array_equal(got[:, j], o.decode(q[:, j], K, V, cut, 0.3))
+    for b in range(B):
+        n = lens[b]
+        qq = torch.from_numpy(np.ascontiguousarray(q[b].transpose(1, 0, 2))).unsqueeze(0)  # [1,H_q,Q,d]
+        kk = torch.from_numpy(np.ascontiguousarray(K[b, :n].transpose(1, 0, 2))).unsqueeze(0)
+        vv = torch.from_numpy(np.ascontiguousarray(V[b, :n].transpose(1, 0, 2))).unsqueeze(0)
+        mask = torch.ones(Q, n, dtype=torch.bool).tril(diagonal=n - Q)
+        ref = F.scaled_dot_product_attention(qq, kk, vv, attn_mask=mask, scale=0.3, enable_gqa=True)
+        assert np.max(np.abs(got[b] - ref[0].transpose(0, 1).numpy())) <= 1e-12
+    _, st = o.decode_multi(q, K, V, np.array([3, 4, 5], dtype=np.int32), 0.3, return_status=True)
+    assert st & 2  # fewer rows than query tokens
+
+
 ALL_PINS = [
     pin_append_position, pin_append_overflow, pin_expand_matches_repeat_interleave,
     pin_single_head_vs_sdpa, pin_decode_vs_sdpa_gqa, pin_mha_endpoint, pin_mqa_endpoint,
     pin_expand_then_attend_equivalence, pin_grouping_changes_output, pin_closed_forms,
     pin_invariants, pin_brute_force_tiny, pin_empty_and_range, pin_divisibility, pin_window,
-    pin_paged,
+    pin_paged, pin_multi_query,
 ]
 
 

@@ -39,6 +39,8 @@ MUTANTS = {
                            "const double *src = pool + ((size_t)page * page_size + t / page_size) * row;"),
     "paged_append_wrong_page": ("int page = block_table[(size_t)b * max_pages + t / page_size];\n        if (page < 0 || page >= n_pages) {\n            if (status) *status |= ORACLE_APPEND_OVERFLOW;",
                                 "int page = block_table[(size_t)b * max_pages + t % page_size];\n        if (page < 0 || page >= n_pages) {\n            if (status) *status |= ORACLE_APPEND_OVERFLOW;"),
+    "multi_not_causal": ("int rows = n - Q + 1 + j;", "int rows = n;"),
+    "multi_off_by_one": ("int rows = n - Q + 1 + j;", "int rows = n - Q + j;"),
     "window_off_by_one": ("int first = (window > 0 && n > window) ? n - window : 0;",
                           "int first = (window > 0 && n > window) ? n - window + 1 : 0;"),
 }
