@@ -182,8 +182,13 @@ def bench_ours(args, rank, world, local):
         caches = [(x["k_cache"].to(dev), x["v_cache"].to(dev))]
     caches.append((caches[0][0].clone(), caches[0][1].clone()))
     lens0 = x["seq_lens_pre"].to(dev)
-    out = torch.empty((w.B, w.H_q, w.d), dtype=torch.float32, device=dev)
-    ws = gqa.alloc_workspace(w.B, w.H_q, w.H_kv, w.d, w.dtype, device=dev)
+    out = torch.empty(tuple(q.shape), dtype=torch.float32, device=dev)
+    if w.queries > 1:
+        nws = gqa.load_library().gqa_decode_multi_workspace_size(w.B, w.queries, w.H_q, w.H_kv, w.d,
+                                                                 gqa.DTYPE_BF16 if w.dtype == torch.bfloat16 else gqa.DTYPE_F32)
+        ws = torch.empty(nws, dtype=torch.uint8, device=dev)
+    else:
+        ws = gqa.alloc_workspace(w.B, w.H_q, w.H_kv, w.d, w.dtype, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
 
     def step(i, lens_row, qq=q, kk=kn, vv=vn):
@@ -192,6 +197,10 @@ def bench_ours(args, rank, world, local):
             gqa.kv_append_paged(kk, vv, kc, vc, block_table, lens_row, status=status)
             gqa.decode_paged(qq, kc, vc, block_table, lens_row, x["scale"], out=out, workspace=ws,
                              status=status)
+            return
+        if w.queries > 1:
+            gqa.kv_append_multi(kk, vv, kc, vc, lens_row, status=status)
+            gqa.decode_multi(qq, kc, vc, lens_row, x["scale"], out=out, workspace=ws, status=status)
             return
         gqa.kv_append(kk, vv, kc, vc, lens_row, status=status)
         if w.window > 0:
@@ -270,7 +279,7 @@ def bench_ours(args, rank, world, local):
     # from pinned host memory and its result out to pinned host memory.
     hq = x["q"].pin_memory()
     hkn, hvn = x["k_new"].pin_memory(), x["v_new"].pin_memory()
-    hout = torch.empty((w.B, w.H_q, w.d), dtype=torch.float32).pin_memory()
+    hout = torch.empty(tuple(q.shape), dtype=torch.float32).pin_memory()
     dq, dkn, dvn = torch.empty_like(q), torch.empty_like(kn), torch.empty_like(vn)
     h2d = hq.numel() * hq.element_size() + 2 * hkn.numel() * hkn.element_size()
     d2h = hout.numel() * 4
@@ -316,7 +325,7 @@ def bench_ours(args, rank, world, local):
             "warmup": W,
             "ms_per_step": round(ms_step, 6),
             "us_per_step": round(ms_step * 1e3, 3),
-            "tokens_per_s": round(w.B * world / (ms_step * 1e-3), 1),
+            "tokens_per_s": round(w.B * w.queries * world / (ms_step * 1e-3), 1),
             "pct_of_measured_hbm": round(100 * value / world / peak, 2),
             "pct_of_8tbs_spec": round(100 * value / world / 8000.0, 2),
             "higher_is_better": True,
@@ -329,6 +338,7 @@ def bench_ours(args, rank, world, local):
                 "L_max": w.L_max, "seq_len": lengths[0] if w.length else "ragged",
                 "window": w.window or None,
                 "page_size": w.page_size or None,
+                "query_tokens": w.queries,
                 "sum_seq_lens": int(sum(lengths)), "kv_dtype": str(w.dtype).replace("torch.", ""),
                 "accumulate": "f32", "ideal_kv_bytes_per_step": ideal,
                 "parallelism": f"replicas x{world}",
@@ -380,11 +390,16 @@ def cpu_baseline(w, x, budget_s, steps=None):
         vc = xb["v_cache"].double().numpy().copy()
         lens = xb["seq_lens_pre"].numpy().copy()
         ts = time.perf_counter()
-        o.kv_append(xb["k_new"].double().numpy(), xb["v_new"].double().numpy(), kc, vc, lens)
-        if w.window > 0:
-            o.decode_window(q, kc, vc, lens, w.window, x["scale"])
+        if w.queries > 1:
+            for j in range(w.queries):  # the Q drafted rows, in order
+                o.kv_append(xb["k_new"][:, j].double().numpy(), xb["v_new"][:, j].double().numpy(), kc, vc, lens)
+            o.decode_multi(q, kc, vc, lens, x["scale"])
         else:
-            o.decode(q, kc, vc, lens, x["scale"])
+            o.kv_append(xb["k_new"].double().numpy(), xb["v_new"].double().numpy(), kc, vc, lens)
+            if w.window > 0:
+                o.decode_window(q, kc, vc, lens, w.window, x["scale"])
+            else:
+                o.decode(q, kc, vc, lens, x["scale"])
         done.append(time.perf_counter() - ts)
         nbytes += inputs.ideal_kv_bytes(w, lens.tolist())
         b = (b + 1) % B

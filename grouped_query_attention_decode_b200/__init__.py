@@ -30,7 +30,8 @@ STATUS_PAGE_RANGE = 16
 # C-ABI symbols declared in include/gqa.h
 EXPORTED = ("gqa_kv_append", "gqa_decode_workspace_size", "gqa_decode", "gqa_status_string",
             "gqa_set_wait_timeout_ns", "gqa_profile_events", "gqa_decode_noalloc",
-            "gqa_decode_window", "gqa_kv_append_paged", "gqa_decode_paged")
+            "gqa_decode_window", "gqa_kv_append_paged", "gqa_decode_paged",
+            "gqa_kv_append_multi", "gqa_decode_multi_workspace_size", "gqa_decode_multi")
 
 
 class GQAError(RuntimeError):
@@ -71,6 +72,14 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gqa_decode_paged.argtypes = [vp, vp, vp, i32p, c_int, i32p, c_int, c_int, c_int, c_int,
                                      c_int, c_int, ctypes.c_float, c_int, vp, vp, c_size, i32p, vp]
     lib.gqa_decode_paged.restype = c_int
+    lib.gqa_kv_append_multi.argtypes = [vp, vp, vp, vp, i32p, c_int, c_int, c_int, c_int, c_int,
+                                        c_int, i32p, vp]
+    lib.gqa_kv_append_multi.restype = c_int
+    lib.gqa_decode_multi_workspace_size.argtypes = [c_int, c_int, c_int, c_int, c_int, c_int]
+    lib.gqa_decode_multi_workspace_size.restype = c_size
+    lib.gqa_decode_multi.argtypes = [vp, vp, vp, i32p, c_int, c_int, c_int, c_int, c_int, c_int,
+                                     ctypes.c_float, c_int, vp, vp, c_size, i32p, vp]
+    lib.gqa_decode_multi.restype = c_int
     lib.gqa_decode_noalloc.argtypes = [vp, vp, vp, i32p, c_int, c_int, c_int, c_int, c_int,
                                        ctypes.c_float, c_int, vp, i32p, vp]
     lib.gqa_decode_noalloc.restype = c_int
@@ -189,6 +198,35 @@ def decode_paged(q, k_pool, v_pool, block_table, seq_lens, scale: float, out=Non
         _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(block_table), max_pages, _ptr(seq_lens), B,
         H_q, H_kv, d, page_size, n_pages, float(scale), _dtype(k_pool), _ptr(out),
         _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream)))
+    return out
+
+
+def kv_append_multi(k_new, v_new, k_cache, v_cache, seq_lens, status=None, stream=None) -> None:
+    """gqa_kv_append_multi: k_new, v_new [B, Q, H_kv, d] to rows seq_lens[b] .. + Q - 1."""
+    B, L_max, H_kv, d = k_cache.shape
+    Q = k_new.shape[1]
+    _check(load_library().gqa_kv_append_multi(
+        _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens), B, Q, H_kv, d,
+        L_max, _dtype(k_cache), _ptr(status), _stream(stream)))
+
+
+def decode_multi(q, k_cache, v_cache, seq_lens, scale: float, out=None, workspace=None,
+                 status=None, stream=None) -> torch.Tensor:
+    """gqa_decode_multi: q [B, Q, H_q, d]; token j attends rows [0, n - Q + 1 + j)."""
+    B, Q, H_q, d = q.shape
+    _, L_max, H_kv, _ = k_cache.shape
+    lib = load_library()
+    if out is None:
+        out = torch.empty((B, Q, H_q, d), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        n = int(lib.gqa_decode_multi_workspace_size(B, Q, H_q, H_kv, d, _DTYPES[k_cache.dtype]))
+        if n == 0:
+            raise GQAError(-9, "no usable sm_100 device is current, or invalid sizes")
+        workspace = torch.empty(n, dtype=torch.uint8, device=q.device)
+    _check(lib.gqa_decode_multi(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens), B, Q, H_q, H_kv, d, L_max,
+        float(scale), _dtype(k_cache), _ptr(out), _ptr(workspace), workspace.numel(),
+        _ptr(status), _stream(stream)))
     return out
 
 

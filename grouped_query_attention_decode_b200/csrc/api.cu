@@ -49,16 +49,19 @@ int current_sm_count(int *dev_out) {
 }
 
 struct Geometry {
-    int r, RB, HB, UB;
+    int r, rb, RB, HB, UB;
     long long units, slots, slot_floats, hdr_floats;
     size_t bytes;
 };
 
-Geometry geometry(int B, int H_q, int H_kv, int d, int G) {
+// Units: (sequence, key/value head, block of rb query heads) with Q query tokens each; a unit
+// has RB = Q * rb <= 64 columns.
+Geometry geometry(int B, int H_q, int H_kv, int d, int G, int Q = 1) {
     Geometry g;
     g.r = H_q / H_kv;
-    g.RB = g.r < 64 ? g.r : 64;
-    g.HB = (g.r + g.RB - 1) / g.RB;
+    g.rb = g.r < 64 / Q ? g.r : 64 / Q;
+    g.RB = Q * g.rb;
+    g.HB = (g.r + g.rb - 1) / g.rb;
     g.UB = H_kv * g.HB;
     g.units = static_cast<long long>(B) * g.UB;
     g.slots = G + g.units - 1;
@@ -114,12 +117,16 @@ bool encode_cache_map(CUtensorMap *m, const void *base, int B, int H_kv, int d, 
                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool encode_q_map(CUtensorMap *m, const void *q, int B, int H_q, int d, int rp) {
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(B) * H_q};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
-    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(rp)};
-    const cuuint32_t estr[2] = {1, 1};
-    return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(q), dims,
+// q as (d, H_q, B*Q); one unit's tile is the box (64 columns, rb heads, Q tokens), which lands
+// in shared memory as rows j * rb + h'.
+bool encode_q_map(CUtensorMap *m, const void *q, int B, int Q, int H_q, int d, int rb) {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H_q),
+                                static_cast<cuuint64_t>(B) * Q};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                                   static_cast<cuuint64_t>(H_q) * d * 2};
+    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(rb), static_cast<cuuint32_t>(Q)};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(q), dims,
                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -144,8 +151,37 @@ extern "C" int gqa_kv_append(const void *k_new, const void *v_new, void *k_cache
     int dev = 0;
     if (current_sm_count(&dev) <= 0) return GQA_ERR_NO_DEVICE;
     const int row_bytes = d * (dtype == GQA_DTYPE_BF16 ? 2 : 4);
-    return launch_append(k_new, v_new, k_cache, v_cache, seq_lens, B, H_kv, row_bytes, L_max,
+    return launch_append(k_new, v_new, k_cache, v_cache, seq_lens, B, H_kv, row_bytes, L_max, 1,
                          status, stream);
+}
+
+extern "C" int gqa_kv_append_multi(const void *k_new, const void *v_new, void *k_cache,
+                                   void *v_cache, int32_t *seq_lens, int B, int Q, int H_kv,
+                                   int d, int L_max, gqa_dtype_t dtype, int32_t *status,
+                                   cudaStream_t stream) {
+    if (!k_new || !v_new || !k_cache || !v_cache || !seq_lens) return GQA_ERR_NULL;
+    if (dtype != GQA_DTYPE_F32 && dtype != GQA_DTYPE_BF16) return GQA_ERR_UNSUPPORTED_DTYPE;
+    if (B <= 0 || Q <= 0 || Q > 64 || H_kv <= 0 || L_max <= 0 ||
+        static_cast<long long>(B) * H_kv > (1ll << 30))
+        return GQA_ERR_SHAPE;
+    if (d != 64 && d != 128) return GQA_ERR_UNSUPPORTED_DIM;
+    if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(k_cache, 16) ||
+        !aligned(v_cache, 16) || !aligned(seq_lens, 4) || (status && !aligned(status, 4)))
+        return GQA_ERR_ALIGNMENT;
+    int dev = 0;
+    if (current_sm_count(&dev) <= 0) return GQA_ERR_NO_DEVICE;
+    const int row_bytes = d * (dtype == GQA_DTYPE_BF16 ? 2 : 4);
+    return launch_append(k_new, v_new, k_cache, v_cache, seq_lens, B, H_kv, row_bytes, L_max, Q,
+                         status, stream);
+}
+
+extern "C" size_t gqa_decode_multi_workspace_size(int B, int Q, int H_q, int H_kv, int d,
+                                                  gqa_dtype_t dtype) {
+    if (Q < 1 || Q > 64 || check_shape(B, H_q, H_kv, d, 1, dtype) != GQA_OK) return 0;
+    int dev = 0;
+    const int sms = current_sm_count(&dev);
+    if (sms <= 0) return 0;
+    return geometry(B, H_q, H_kv, d, sms, Q).bytes;
 }
 
 extern "C" size_t gqa_decode_workspace_size(int B, int H_q, int H_kv, int d, gqa_dtype_t dtype) {
@@ -167,7 +203,8 @@ struct PagedArgs {
 int decode_impl(const void *q, const void *k_cache, const void *v_cache, const int32_t *seq_lens,
                 int B, int H_q, int H_kv, int d, int L_max, int window, float scale,
                 gqa_dtype_t dtype, float *out, void *workspace, size_t workspace_bytes,
-                int32_t *status, cudaStream_t stream, const PagedArgs &pg = PagedArgs()) {
+                int32_t *status, cudaStream_t stream, const PagedArgs &pg = PagedArgs(),
+                int Q = 1) {
     if (!q || !k_cache || !v_cache || !seq_lens || !out) return GQA_ERR_NULL;
     const int rc = check_shape(B, H_q, H_kv, d, L_max, dtype);
     if (rc != GQA_OK) return rc;
@@ -179,7 +216,8 @@ int decode_impl(const void *q, const void *k_cache, const void *v_cache, const i
     int dev = 0;
     const int sms = current_sm_count(&dev);
     if (sms <= 0) return GQA_ERR_NO_DEVICE;
-    const Geometry g = geometry(B, H_q, H_kv, d, sms);
+    if (Q < 1 || Q > 64) return GQA_ERR_SHAPE;
+    const Geometry g = geometry(B, H_q, H_kv, d, sms, Q);
     if (workspace_bytes < g.bytes) return GQA_ERR_WORKSPACE;
 
     DecodeParams p;
@@ -193,6 +231,9 @@ int decode_impl(const void *q, const void *k_cache, const void *v_cache, const i
     p.d = d;
     p.L_max = L_max;
     p.r = g.r;
+    p.Q = Q;
+    p.rb = g.rb;
+    p.q_box_bytes = (d / 64) * Q * g.rb * 128;
     p.RB = g.RB;
     p.HB = g.HB;
     p.UB = g.UB;
@@ -223,7 +264,8 @@ int decode_impl(const void *q, const void *k_cache, const void *v_cache, const i
         const int rows_dim = pg.block_table ? pg.page_size : L_max;
         const int outer_dim = pg.block_table ? pg.n_pages : B;
         const int box = pg.block_table ? (pg.page_size < 128 ? pg.page_size : 128) : 128;
-        if (!encode_q_map(&maps.q, q, B, H_q, d, rp) ||
+        (void)rp;
+        if (!encode_q_map(&maps.q, q, B, Q, H_q, d, g.rb) ||
             !encode_cache_map(&maps.k, k_cache, outer_dim, H_kv, d, rows_dim, box) ||
             !encode_cache_map(&maps.k8, k_cache, outer_dim, H_kv, d, rows_dim, 8) ||
             !encode_cache_map(&maps.v, v_cache, outer_dim, H_kv, d, rows_dim, box) ||
@@ -294,6 +336,16 @@ extern "C" int gqa_decode_paged(const void *q, const void *k_pool, const void *v
     pg.n_pages = n_pages;
     return decode_impl(q, k_pool, v_pool, seq_lens, B, H_q, H_kv, d, max_pages * page_size, 0,
                        scale, dtype, out, workspace, workspace_bytes, status, stream, pg);
+}
+
+extern "C" int gqa_decode_multi(const void *q, const void *k_cache, const void *v_cache,
+                                const int32_t *seq_lens, int B, int Q, int H_q, int H_kv, int d,
+                                int L_max, float scale, gqa_dtype_t dtype, float *out,
+                                void *workspace, size_t workspace_bytes, int32_t *status,
+                                cudaStream_t stream) {
+    if (Q < 1 || Q > 64) return GQA_ERR_SHAPE;
+    return decode_impl(q, k_cache, v_cache, seq_lens, B, H_q, H_kv, d, L_max, 0, scale, dtype,
+                       out, workspace, workspace_bytes, status, stream, PagedArgs(), Q);
 }
 
 extern "C" int gqa_decode_window(const void *q, const void *k_cache, const void *v_cache,

@@ -11,29 +11,32 @@
 
 namespace gqa {
 
+// Appends `rows` consecutive rows per sequence (rows = 1 for one decode step; several for the
+// drafted tokens of a speculative step), which form one contiguous block of the cache.
 __global__ void __launch_bounds__(128)
 append_kernel(const uint4 *__restrict__ k_new, const uint4 *__restrict__ v_new, uint4 *k_cache,
-              uint4 *v_cache, int32_t *seq_lens, int H_kv, int row_vecs, int L_max,
+              uint4 *v_cache, int32_t *seq_lens, int H_kv, int row_vecs, int L_max, int rows,
               int32_t *status) {
     const int b = blockIdx.x;
     const int t = seq_lens[b];
     // Let a following decode launch start its prologue while this copy runs.
     grid_launch_dependents();
     __syncthreads();  // every thread has read seq_lens[b] before thread 0 advances it
-    if (t < 0 || t >= L_max) {
+    if (t < 0 || t > L_max - rows) {
         if (threadIdx.x == 0 && status != nullptr) atomicOr(status, GQA_STATUS_APPEND_OVERFLOW);
         return;
     }
-    const long long blk = static_cast<long long>(H_kv) * row_vecs;  // 16-byte vectors per row block
+    const long long row = static_cast<long long>(H_kv) * row_vecs;  // 16-byte vectors per row
+    const long long blk = row * rows;
     const uint4 *ks = k_new + b * blk;
     const uint4 *vs = v_new + b * blk;
-    uint4 *kd = k_cache + (static_cast<long long>(b) * L_max + t) * blk;
-    uint4 *vd = v_cache + (static_cast<long long>(b) * L_max + t) * blk;
+    uint4 *kd = k_cache + (static_cast<long long>(b) * L_max + t) * row;
+    uint4 *vd = v_cache + (static_cast<long long>(b) * L_max + t) * row;
     for (long long i = threadIdx.x; i < blk; i += blockDim.x) {
         kd[i] = ks[i];
         vd[i] = vs[i];
     }
-    if (threadIdx.x == 0) seq_lens[b] = t + 1;
+    if (threadIdx.x == 0) seq_lens[b] = t + rows;
 }
 
 // Paged variant: row t = seq_lens[b] goes to row t % page_size of page
@@ -80,12 +83,12 @@ int launch_append_paged(const void *k_new, const void *v_new, void *k_pool, void
 }
 
 int launch_append(const void *k_new, const void *v_new, void *k_cache, void *v_cache,
-                  int32_t *seq_lens, int B, int H_kv, int row_bytes, int L_max, int32_t *status,
-                  cudaStream_t stream) {
+                  int32_t *seq_lens, int B, int H_kv, int row_bytes, int L_max, int rows,
+                  int32_t *status, cudaStream_t stream) {
     append_kernel<<<B, 128, 0, stream>>>(
         static_cast<const uint4 *>(k_new), static_cast<const uint4 *>(v_new),
         static_cast<uint4 *>(k_cache), static_cast<uint4 *>(v_cache), seq_lens, H_kv,
-        row_bytes / 16, L_max, status);
+        row_bytes / 16, L_max, rows, status);
     return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 

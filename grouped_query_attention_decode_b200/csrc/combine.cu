@@ -33,18 +33,19 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const DecodePa
     const int k = u - b * p.UB;
     const int kvh = k / p.HB;
     const int hb = k - kvh * p.HB;
-    const int nh = min(p.RB, p.r - hb * p.RB);
-    const int h0 = kvh * p.r + hb * p.RB;
+    const int nh = p.RB;  // columns of the unit (and slot layout stride)
     const int d = p.d;
     const int first = blockIdx.y * kCombineOutputsPerCta;
     const int last = min(nh * d, first + kCombineOutputsPerCta);
     if (first >= last) return;
-    float *o = p.out + (static_cast<long long>(b) * p.H_q + h0) * d;
     const long long *hdr = reinterpret_cast<const long long *>(p.ws);
-    const int n = valid_len(p.seq_lens[b], p.L_max);
+    const int n = valid_len(p.seq_lens[b], p.L_max, p.Q);
     const int nt = seq_tiles(n, p);
     if (nt == 0) {
-        for (int idx = first + threadIdx.x; idx < last; idx += blockDim.x) o[idx] = 0.f;
+        for (int idx = first + threadIdx.x; idx < last; idx += blockDim.x) {
+            const long long orow = out_row(p, b, kvh, hb, idx / d);
+            if (orow >= 0) p.out[orow * d + idx % d] = 0.f;
+        }
         return;
     }
     const long long total = hdr[p.B];
@@ -90,11 +91,13 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const DecodePa
     __syncthreads();
     for (int idx = first + threadIdx.x; idx < last; idx += blockDim.x) {
         const int h = idx / d;
+        const long long orow = out_row(p, b, kvh, hb, h);
+        if (orow < 0) continue;
         float acc = 0.f;
 #pragma unroll 4
         for (int c = 0; c < np; ++c)
             acc = fmaf(wts[c * nh + h], slots[static_cast<long long>(piece_cta[c]) * p.slot_floats + idx], acc);
-        o[idx] = acc;
+        p.out[orow * d + (idx - h * d)] = acc;
     }
 }
 

@@ -69,10 +69,12 @@ split_f32_kernel(const float *__restrict__ q, const float *__restrict__ kc,
     Segment sg;
     constexpr int ACC = C::RBMAX * D / 256;
     while (w.next(sg)) {
-        const int nh = min(p.RB, p.r - sg.hb * p.RB);
-        const int h0 = sg.kvh * p.r + sg.hb * p.RB;
-        const float *qrow = q + (static_cast<long long>(sg.b) * p.H_q + h0) * D;
-        for (int idx = tid; idx < nh * D; idx += 256) qs[idx] = qrow[idx];
+        // columns of the unit: (token j, head h') pairs, j * rb + h'
+        const int nh = p.RB;
+        for (int idx = tid; idx < nh * D; idx += 256) {
+            const long long qr = out_row(p, sg.b, sg.kvh, sg.hb, idx / D);  // same row layout as out
+            qs[idx] = qr >= 0 ? q[qr * D + idx % D] : 0.f;
+        }
         if (tid < nh) {
             ms[tid] = -INFINITY;
             ls[tid] = 0.f;
@@ -110,7 +112,8 @@ split_f32_kernel(const float *__restrict__ q, const float *__restrict__ kc,
                 const int h = idx / T;
                 const int t = idx - h * T;
                 float s = -INFINITY;
-                if (t < rows) {
+                // token j = h / rb of the unit sees rows < n - Q + 1 + j
+                if (t < rows && row0 + t < sg.n - p.Q + 1 + h / p.rb) {
                     const float4 *qa = reinterpret_cast<const float4 *>(qs + h * D);
                     const float4 *ka = reinterpret_cast<const float4 *>(ks + t * KP);
                     float a = 0.f;
@@ -132,8 +135,11 @@ split_f32_kernel(const float *__restrict__ q, const float *__restrict__ kc,
                 const float tmax = warp_max_f32(fmaxf(a, b));
                 const float m_old = ms[h];
                 const float m_new = fmaxf(m_old, tmax);
-                const float alpha = ex2_approx(m_old - m_new);
-                const float pa = ex2_approx(a - m_new), pb = ex2_approx(b - m_new);
+                // no visible row yet (several query tokens): nothing to rescale or add
+                const bool none = m_new == -INFINITY;
+                const float alpha = none ? 1.f : ex2_approx(m_old - m_new);
+                const float pa = a == -INFINITY ? 0.f : ex2_approx(a - m_new);
+                const float pb = b == -INFINITY ? 0.f : ex2_approx(b - m_new);
                 ss[h * T + lane] = pa;
                 ss[h * T + lane + 32] = pb;
                 const float sum = warp_sum_f32(pa + pb);
@@ -159,11 +165,13 @@ split_f32_kernel(const float *__restrict__ q, const float *__restrict__ kc,
             __syncthreads();
         }
         if (sg.whole) {
-            float *o = p.out + (static_cast<long long>(sg.b) * p.H_q + h0) * D;
 #pragma unroll
             for (int k = 0; k < ACC; ++k) {
                 const int idx = tid + 256 * k;
-                if (idx < nh * D) o[idx] = acc[k] / ls[idx / D];
+                if (idx < nh * D) {
+                    const long long orow = out_row(p, sg.b, sg.kvh, sg.hb, idx / D);
+                    if (orow >= 0) p.out[orow * D + idx % D] = acc[k] / ls[idx / D];
+                }
             }
         } else {
             float *slot = p.ws + p.hdr_floats + (static_cast<long long>(blockIdx.x) + sg.unit) * p.slot_floats;

@@ -164,6 +164,10 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         sm->abort = 0;
         fence_mbarrier_init();
     }
+    // q rows past a unit's columns are never loaded: zero them once so padded columns see zeros
+    for (int c = threadIdx.x; c < C::QB * C::Q_BYTES / 16; c += C::THREADS)
+        reinterpret_cast<uint4 *>(q_base)[c] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
     if (warp == 0) {
         tmem_alloc(&sm->tmem_base, C::TMEM_COLS);
         tmem_relinquish();
@@ -222,12 +226,12 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     ok = false;
                     break;
                 }
-                mbar_arrive_expect_tx(&sm->q_full[qb], C::Q_BYTES);
-                const int qrow = sg.b * p.H_q + sg.kvh * p.r + sg.hb * p.RB;
+                // q of the unit: rows (token j, head h') of q viewed as (d, H_q, B*Q)
+                mbar_arrive_expect_tx(&sm->q_full[qb], p.q_box_bytes);
 #pragma unroll
                 for (int kb = 0; kb < C::KB; ++kb)
-                    tma_load_2d(q_base + qb * C::Q_BYTES + kb * RP * 128, &tm_q, &sm->q_full[qb],
-                                kb * 64, qrow);
+                    tma_load_3d(q_base + qb * C::Q_BYTES + kb * RP * 128, &tm_q, &sm->q_full[qb],
+                                kb * 64, sg.kvh * p.r + sg.hb * p.rb, sg.b * p.Q);
                 ++sidx;
                 for (int jj = 0; jj < sg.len; ++jj) {
                     const int st = i % S;
@@ -415,8 +419,6 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         bool ok = true;
         float O[NHW], l[NHW], m_run[NHW], alpha[NHW];
         while (ok && w.next(sg)) {
-            const int nh = min(p.RB, p.r - sg.hb * p.RB);
-            const int nhw = min(NHW, max(0, nh - hbase));  // this group's real heads
 #pragma unroll
             for (int h = 0; h < NHW; ++h) {
                 O[h] = 0.f;
@@ -458,10 +460,14 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
 
                 const bool valid = row < rows;
+                // Several query tokens: column j * rb + h' sees rows < n - Q + 1 + j, so a row
+                // `over` rows past n - Q is visible only to columns >= (over + 1) * rb.
+                const int over = sg.first + (sg.j0 + jj) * T + row - (sg.n - p.Q + 1);
+                const int min_col = over >= 0 ? (over + 1) * p.rb : 0;
                 float x[NHW];
 #pragma unroll
                 for (int h = 0; h < NHW; ++h)
-                    x[h] = valid ? __uint_as_float(sr[h]) * p.scale_log2 : -INFINITY;
+                    x[h] = (valid && hbase + h >= min_col) ? __uint_as_float(sr[h]) * p.scale_log2 : -INFINITY;
                 // Per-head maximum over the warp's 32 rows.
                 {
                     float wm[NHW];
@@ -506,7 +512,9 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     constexpr int HALF_VALS = C::P_ROWB / 2;  // bf16 values per atom row
 #pragma unroll
                     for (int h = 0; h < NHW; ++h) {
-                        x[h] = ex2_approx(x[h] - m_run[h]);  // x now holds p
+                        // x now holds p; a column with no visible row yet (several query tokens)
+                        // keeps p = 0 rather than exp(-inf + inf)
+                        x[h] = x[h] == -INFINITY ? 0.f : ex2_approx(x[h] - m_run[h]);
                         l[h] = l[h] * alpha[h] + x[h];
                     }
 #pragma unroll
@@ -592,30 +600,30 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 break;
             }
             if (dcol >= 0) {
-                const int h0 = sg.kvh * p.r + sg.hb * p.RB + hbase;
                 if (sg.whole) {
-                    float *o = p.out + (static_cast<long long>(sg.b) * p.H_q + h0) * D + dcol;
 #pragma unroll
                     for (int h = 0; h < NHW; ++h) {
-                        if (h < nhw) {
+                        const long long orow = out_row(p, sg.b, sg.kvh, sg.hb, hbase + h);
+                        if (orow >= 0) {
                             const float L = sm->lsum[wg][0][h] + sm->lsum[wg][1][h] + sm->lsum[wg][2][h] + sm->lsum[wg][3][h];
-                            o[static_cast<long long>(h) * D] = O[h] / L;
+                            p.out[orow * D + dcol] = O[h] / L;
                         }
                     }
                 } else {
+                    // slot: O [RB][D], then m [RB], then l [RB] (padding columns included)
                     float *slot = p.ws + p.hdr_floats +
                                   (static_cast<long long>(blockIdx.x) + sg.unit) * p.slot_floats;
 #pragma unroll
                     for (int h = 0; h < NHW; ++h)
-                        if (h < nhw) slot[(hbase + h) * D + dcol] = O[h];
-                    if (dcol < nhw) {
+                        if (hbase + h < p.RB) slot[(hbase + h) * D + dcol] = O[h];
+                    if (dcol < NHW && hbase + dcol < p.RB) {
                         const int h = dcol;
                         float m_final = -INFINITY;
 #pragma unroll
                         for (int hh = 0; hh < NHW; ++hh)
                             if (hh == h) m_final = m_run[hh];
-                        slot[nh * D + hbase + h] = m_final;
-                        slot[nh * D + nh + hbase + h] = sm->lsum[wg][0][h] + sm->lsum[wg][1][h] + sm->lsum[wg][2][h] + sm->lsum[wg][3][h];
+                        slot[p.RB * D + hbase + h] = m_final;
+                        slot[p.RB * D + p.RB + hbase + h] = sm->lsum[wg][0][h] + sm->lsum[wg][1][h] + sm->lsum[wg][2][h] + sm->lsum[wg][3][h];
                     }
                 }
             }

@@ -26,7 +26,7 @@ int launch_append_paged(const void *k_new, const void *v_new, void *k_pool, void
                         int H_kv, int row_bytes, int page_size, int n_pages, int32_t *status,
                         cudaStream_t stream);
 int launch_append(const void *k_new, const void *v_new, void *k_cache, void *v_cache,
-                  int32_t *seq_lens, int B, int H_kv, int row_bytes, int L_max, int32_t *status,
-                  cudaStream_t stream);
+                  int32_t *seq_lens, int B, int H_kv, int row_bytes, int L_max, int rows,
+                  int32_t *status, cudaStream_t stream);
 
 }  // namespace gqa

@@ -27,8 +27,11 @@ struct DecodeParams {
     int32_t *status;          // device status word or nullptr
     int B, H_q, H_kv, d, L_max;
     int r;     // query heads per key/value head
-    int RB;    // query heads per unit (<= 64)
-    int HB;    // units per key/value head = ceil(r / RB)
+    int Q;     // query tokens per sequence (1, or several for speculative verification)
+    int rb;    // query heads per unit and token; a unit's columns are (token j, head h') pairs
+    int RB;    // columns per unit = Q * rb (<= 64), column index j * rb + h'
+    int HB;    // units per key/value head = ceil(r / rb)
+    int q_box_bytes;  // bytes of the q tile of one unit (bf16 path)
     int UB;    // units per sequence = H_kv * HB
     int T;     // cached rows per tile
     int G;     // CTAs of the split kernel
@@ -44,8 +47,19 @@ struct DecodeParams {
     long long hdr_floats;             // header length in floats (int64 offsets [B + 1])
 };
 
-__device__ __forceinline__ int valid_len(int n, int L_max) {
-    return (n < 0 || n > L_max) ? 0 : n;
+// Row of out [B*Q][H_q] that unit column hh (token hh / rb, head hh % rb) writes, or -1 for a
+// padding column (past the group's heads in the last head block).
+__device__ __forceinline__ long long out_row(const DecodeParams &p, int b, int kvh, int hb, int hh) {
+    const int j = hh / p.rb, hp = hh - j * p.rb;
+    const int nhb = min(p.rb, p.r - hb * p.rb);
+    if (j >= p.Q || hp >= nhb) return -1;
+    return (static_cast<long long>(b) * p.Q + j) * p.H_q + kvh * p.r + hb * p.rb + hp;
+}
+
+// Rows a sequence of length n may attend: n, or 0 when n is out of range -- negative, past
+// L_max, or (several query tokens) shorter than the Q tokens that must be in the cache.
+__device__ __forceinline__ int valid_len(int n, int L_max, int Q) {
+    return (n < 0 || n > L_max || (Q > 1 && n < Q)) ? 0 : n;
 }
 
 __device__ __forceinline__ int tiles_of(int n, int T) { return (n + T - 1) / T; }
@@ -95,7 +109,7 @@ __device__ inline CtaRange locate_cta_range(const DecodeParams &p, int cta, int 
         int n = 0;
         if (b < p.B) {
             const int raw = p.seq_lens[b];
-            n = valid_len(raw, p.L_max);
+            n = valid_len(raw, p.L_max, p.Q);
             if (flag_range && n != raw && p.status != nullptr) atomicOr(p.status, GQA_STATUS_SEQLEN_RANGE);
         }
         const long long v = static_cast<long long>(seq_tiles(n, p)) * p.UB;
@@ -114,7 +128,7 @@ __device__ inline CtaRange locate_cta_range(const DecodeParams &p, int cta, int 
     long long off = 0;
     for (int base = 0; base < p.B; base += 32) {
         const int b = base + lane;
-        const int n = b < p.B ? valid_len(p.seq_lens[b], p.L_max) : 0;
+        const int n = b < p.B ? valid_len(p.seq_lens[b], p.L_max, p.Q) : 0;
         const long long v = static_cast<long long>(seq_tiles(n, p)) * p.UB;
         const long long incl = warp_incl_scan(v, lane);
         const long long excl = incl - v;
@@ -145,7 +159,7 @@ struct Segment {
 // all of them see the same sequence of segments.
 struct SegmentWalker {
     const int32_t *lens;
-    int B, UB, HB, L_max, T, window;
+    int B, UB, HB, L_max, T, window, Q;
     int b, n, nt;
     long long off, t, end;
 
@@ -157,12 +171,13 @@ struct SegmentWalker {
         L_max = p.L_max;
         T = p.T;
         window = p.window;
+        Q = p.Q;
         t = cr.begin;
         end = cr.end;
         b = cr.b0;
         off = cr.off0;
         if (t < end) {
-            n = valid_len(lens[b], L_max);
+            n = valid_len(lens[b], L_max, Q);
             nt = tiles_of(n - first_row(n, window), T);
         } else {
             n = 0;
@@ -178,7 +193,7 @@ struct SegmentWalker {
                 t = end;
                 return false;
             }
-            n = valid_len(lens[b], L_max);
+            n = valid_len(lens[b], L_max, Q);
             nt = tiles_of(n - first_row(n, window), T);
         }
         const long long rel = t - off;

@@ -12,7 +12,9 @@ Recipe (all draws from one ``torch.Generator('cpu')`` seeded with the workload's
   6. lengths  [B]  either the fixed length, or uniform integers in [1, L_max] (ragged)
 Each float is drawn in fp32 and rounded to the storage dtype with round-to-nearest-even.
 ``lengths`` is the number of rows attended AFTER this step's append, so the cache starts with
-``seq_lens = lengths - 1`` and the append writes row ``lengths - 1``.  Cache rows at or beyond
+``seq_lens = lengths - 1`` and the append writes row ``lengths - 1``.  With Q > 1 query tokens
+per sequence (speculative verification), q is [B, Q, H_q, d], k_new/v_new are [B, Q, H_kv, d]
+and the append writes the last Q rows.  Cache rows at or beyond
 ``lengths - 1`` hold no data the step may read; ``poison=True`` fills them with NaN so a kernel
 that reads them poisons its output.
 """
@@ -40,6 +42,7 @@ class Workload:
     scale: float | None = None         # None = 1/sqrt(d)
     window: int = 0                    # > 0: sliding window, attend the last `window` rows
     page_size: int = 0                 # > 0: the cache lives in a paged pool (see make_paged)
+    queries: int = 1                   # query tokens per sequence (speculative verification)
     note: str = field(default="", compare=False)
 
     @property
@@ -78,6 +81,9 @@ WORKLOADS = {
         Workload("llama2_70b_layer_paged16", B=16, H_q=64, H_kv=8, d=128, L_max=4096,
                  dtype=torch.bfloat16, q_std=0.5, kv_std=0.5, seed=1, length=4096, page_size=16,
                  note="the Llama-2-70B-shaped layer in a paged pool of 16-row pages"),
+        Workload("llama2_70b_layer_spec4", B=16, H_q=64, H_kv=8, d=128, L_max=4096,
+                 dtype=torch.bfloat16, q_std=0.5, kv_std=0.5, seed=1, length=4096, queries=4,
+                 note="the Llama-2-70B-shaped layer verifying 4 drafted tokens per sequence"),
         Workload("ragged_long_window4096", B=32, H_q=32, H_kv=8, d=128, L_max=32768,
                  dtype=torch.bfloat16, q_std=1.0, kv_std=1.0, seed=4, length=None, window=4096,
                  note="the ragged batch with a Mistral-style sliding window of 4096 rows"),
@@ -86,10 +92,11 @@ WORKLOADS = {
 
 
 def custom(name="custom", *, B, H_q, H_kv, d, L_max, dtype=torch.bfloat16, q_std=1.0,
-           kv_std=1.0, seed=1234, length=None, scale=None, window=0, page_size=0) -> Workload:
+           kv_std=1.0, seed=1234, length=None, scale=None, window=0, page_size=0,
+           queries=1) -> Workload:
     return Workload(name, B=B, H_q=H_q, H_kv=H_kv, d=d, L_max=L_max, dtype=dtype, q_std=q_std,
                     kv_std=kv_std, seed=seed, length=length, scale=scale, window=window,
-                    page_size=page_size)
+                    page_size=page_size, queries=queries)
 
 
 def _normal(shape, gen, std, dtype):
@@ -108,15 +115,17 @@ def make_inputs(w: Workload, lengths=None, poison: bool = False) -> dict:
     """
     g = torch.Generator(device="cpu")
     g.manual_seed(w.seed)
-    q = _normal((w.B, w.H_q, w.d), g, w.q_std, w.dtype)
+    Qn = w.queries
+    q = _normal((w.B, w.H_q, w.d) if Qn == 1 else (w.B, Qn, w.H_q, w.d), g, w.q_std, w.dtype)
     k_cache = torch.empty((w.B, w.L_max, w.H_kv, w.d), dtype=w.dtype)
     v_cache = torch.empty_like(k_cache)
     for b in range(w.B):
         k_cache[b] = _normal((w.L_max, w.H_kv, w.d), g, w.kv_std, w.dtype)
     for b in range(w.B):
         v_cache[b] = _normal((w.L_max, w.H_kv, w.d), g, w.kv_std, w.dtype)
-    k_new = _normal((w.B, w.H_kv, w.d), g, w.kv_std, w.dtype)
-    v_new = _normal((w.B, w.H_kv, w.d), g, w.kv_std, w.dtype)
+    new_shape = (w.B, w.H_kv, w.d) if Qn == 1 else (w.B, Qn, w.H_kv, w.d)
+    k_new = _normal(new_shape, g, w.kv_std, w.dtype)
+    v_new = _normal(new_shape, g, w.kv_std, w.dtype)
     if w.length is not None:
         drawn = torch.full((w.B,), w.length, dtype=torch.int32)
     else:
@@ -124,7 +133,7 @@ def make_inputs(w: Workload, lengths=None, poison: bool = False) -> dict:
     if lengths is not None:
         drawn = torch.tensor(list(lengths), dtype=torch.int32)
         assert drawn.shape == (w.B,)
-    seq_lens_pre = torch.clamp(drawn - 1, min=0).to(torch.int32)
+    seq_lens_pre = torch.clamp(drawn - Qn, min=0).to(torch.int32)
     if poison:
         nan = float("nan")
         for b in range(w.B):

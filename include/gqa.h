@@ -150,6 +150,30 @@ int gqa_decode_window(const void *q, const void *k_cache, const void *v_cache,
                       size_t workspace_bytes, int32_t *status, cudaStream_t stream);
 
 /*
+ * Several query tokens per sequence (speculative decoding).  "GQA 阅读笔记", what came after GQA
+ * and the engineering notes on speculative decoding: when the target model checks k drafted
+ * tokens in one pass, the cache is read once and all k new queries attend it.  With Q tokens
+ * per sequence, the Q new tokens are the last Q rows of the cache and token j (0 <= j < Q)
+ * attends rows [0, n - Q + 1 + j) of its sequence, n = seq_lens[b] (causal among the drafts;
+ * Q = 1 is gqa_decode).  Each cached K/V row is read once for all Q tokens and all r heads.
+ *
+ * gqa_kv_append_multi: append Q rows per sequence: k_new, v_new [B][Q][H_kv][d] go to rows
+ *   t .. t+Q-1, t = seq_lens[b]; then seq_lens[b] = t + Q.  t + Q > L_max (or t < 0) is
+ *   refused with GQA_STATUS_APPEND_OVERFLOW.
+ * gqa_decode_multi: q [B][Q][H_q][d] -> out [B][Q][H_q][d] (float32); seq_lens[b] >= Q, else
+ *   out[b] = 0 and GQA_STATUS_SEQLEN_RANGE.  1 <= Q <= 64.  The workspace is
+ *   gqa_decode_multi_workspace_size(B, Q, ...) bytes.  Other arguments as gqa_decode.
+ */
+int gqa_kv_append_multi(const void *k_new, const void *v_new, void *k_cache, void *v_cache,
+                        int32_t *seq_lens, int B, int Q, int H_kv, int d, int L_max,
+                        gqa_dtype_t dtype, int32_t *status, cudaStream_t stream);
+size_t gqa_decode_multi_workspace_size(int B, int Q, int H_q, int H_kv, int d, gqa_dtype_t dtype);
+int gqa_decode_multi(const void *q, const void *k_cache, const void *v_cache,
+                     const int32_t *seq_lens, int B, int Q, int H_q, int H_kv, int d, int L_max,
+                     float scale, gqa_dtype_t dtype, float *out, void *workspace,
+                     size_t workspace_bytes, int32_t *status, cudaStream_t stream);
+
+/*
  * Paged KV cache.  "GQA 阅读笔记", section on what came after GQA (the vLLM PagedAttention
  * paragraph: the KV cache is managed in fixed-size blocks) and "GQA 深入理解", section 8
  * (PagedAttention organises the cache to cut fragmentation).  All sequences share one pool
