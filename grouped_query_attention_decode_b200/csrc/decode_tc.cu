@@ -32,6 +32,8 @@
 namespace gqa {
 
 constexpr unsigned long long kDrainNs = 1000000000ull;  // bound for draining in-flight work
+// Scores may exceed the running maximum by this much (log2 units) before it is raised.
+constexpr float kLazyLog2 = 8.0f;
 
 template <int D, int NH>
 struct TcCfg {
@@ -468,39 +470,51 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                 for (int h = 0; h < NHW; ++h)
                     x[h] = (valid && hbase + h >= min_col) ? __uint_as_float(sr[h]) * p.scale_log2 : -INFINITY;
-                // Per-head maximum over the warp's 32 rows.
-                {
-                    float wm[NHW];
+                // Lazy rescaling.  The running maximum m_run only has to keep the exponents in
+                // range, so it is raised -- through an exchange of the warps' tile maxima -- only
+                // when some score of the tile exceeds it by more than kLazyLog2; otherwise every
+                // p = 2^(x - m_run) <= 2^kLazyLog2 and nothing is rescaled.  The result is exact
+                // either way: P, the running sums and O always share one reference.
+                bool need = false;
 #pragma unroll
-                    for (int h = 0; h < NHW; ++h) wm[h] = x[h];
-                    warp_max_transpose<NHW, C::LOG2NHW>(wm, lane);
-                    if (lane < NHW)
-                        reinterpret_cast<float *>(&sm->wmax[wg][j2][q4][0])[transpose_head<NHW, C::LOG2NHW>(lane)] = wm[0];
-                }
-                if (named_bar_any(bar_id, 128, bad)) {
-                    ok = false;
-                    break;
-                }
-                // Every thread forms the tile maximum of each of its heads from the four warp
-                // maxima and keeps the running maximum in registers (identical in all threads
-                // of the group), so one barrier per tile suffices.
+                for (int h = 0; h < NHW; ++h) need |= x[h] > m_run[h] + kLazyLog2;
+                if (named_bar_any(bar_id, 128, bad || need)) {
+                    // Per-head maximum over the warp's 32 rows, then over the four warps.
+                    {
+                        float wm[NHW];
 #pragma unroll
-                for (int h4 = 0; h4 < C::NHW4; ++h4) {
-                    const float4 a = sm->wmax[wg][j2][0][h4], b = sm->wmax[wg][j2][1][h4];
-                    const float4 c = sm->wmax[wg][j2][2][h4], e = sm->wmax[wg][j2][3][h4];
-                    const float t4[4] = {fmaxf(fmaxf(a.x, b.x), fmaxf(c.x, e.x)),
-                                         fmaxf(fmaxf(a.y, b.y), fmaxf(c.y, e.y)),
-                                         fmaxf(fmaxf(a.z, b.z), fmaxf(c.z, e.z)),
-                                         fmaxf(fmaxf(a.w, b.w), fmaxf(c.w, e.w))};
+                        for (int h = 0; h < NHW; ++h) wm[h] = x[h];
+                        warp_max_transpose<NHW, C::LOG2NHW>(wm, lane);
+                        if (lane < NHW)
+                            reinterpret_cast<float *>(&sm->wmax[wg][j2][q4][0])[transpose_head<NHW, C::LOG2NHW>(lane)] = wm[0];
+                    }
+                    if (named_bar_any(bar_id, 128, bad)) {
+                        ok = false;
+                        break;
+                    }
+                    // Every thread forms the tile maximum of each of its heads from the four
+                    // warp maxima; the running maximum stays identical in all threads.
 #pragma unroll
-                    for (int e4 = 0; e4 < 4; ++e4) {
-                        const int h = h4 * 4 + e4;
-                        if (h < NHW) {
-                            const float m_new = fmaxf(m_run[h], t4[e4]);
-                            alpha[h] = m_new == -INFINITY ? 0.f : ex2_approx(m_run[h] - m_new);
-                            m_run[h] = m_new;
+                    for (int h4 = 0; h4 < C::NHW4; ++h4) {
+                        const float4 a = sm->wmax[wg][j2][0][h4], b = sm->wmax[wg][j2][1][h4];
+                        const float4 c = sm->wmax[wg][j2][2][h4], e = sm->wmax[wg][j2][3][h4];
+                        const float t4[4] = {fmaxf(fmaxf(a.x, b.x), fmaxf(c.x, e.x)),
+                                             fmaxf(fmaxf(a.y, b.y), fmaxf(c.y, e.y)),
+                                             fmaxf(fmaxf(a.z, b.z), fmaxf(c.z, e.z)),
+                                             fmaxf(fmaxf(a.w, b.w), fmaxf(c.w, e.w))};
+#pragma unroll
+                        for (int e4 = 0; e4 < 4; ++e4) {
+                            const int h = h4 * 4 + e4;
+                            if (h < NHW) {
+                                const float m_new = fmaxf(m_run[h], t4[e4]);
+                                alpha[h] = m_new == -INFINITY ? 0.f : ex2_approx(m_run[h] - m_new);
+                                m_run[h] = m_new;
+                            }
                         }
                     }
+                } else {
+#pragma unroll
+                    for (int h = 0; h < NHW; ++h) alpha[h] = 1.f;
                 }
 
                 // P = hi + lo in bf16 (~16 significant bits).  This thread's tile row is K row

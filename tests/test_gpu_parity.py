@@ -166,3 +166,26 @@ def test_deterministic():
     a, _, _, _ = run_step(x)
     b, _, _, _ = run_step(x)
     assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("pattern", ["growing", "jump", "shrinking"])
+def test_running_max_paths(oracle, pattern):
+    """The running maximum is raised only when a tile's scores exceed it by more than a margin;
+    scores that grow along the sequence, jump once by far more than the margin, or start high and
+    shrink exercise both the lazy path and the rescaling path."""
+    w = inputs.custom("maxpath", B=3, H_q=16, H_kv=2, d=128, L_max=1500, dtype=torch.bfloat16,
+                      q_std=0.5, kv_std=1.0, seed=33)
+    x = inputs.make_inputs(w, lengths=[1500, 700, 300])
+    t = torch.arange(w.L_max, dtype=torch.float32)
+    if pattern == "growing":
+        f = 1.0 + 6.0 * t / w.L_max
+    elif pattern == "jump":
+        f = torch.where(t < 600, torch.full_like(t, 0.3), torch.full_like(t, 6.0))
+    else:
+        f = 6.0 - 5.0 * t / w.L_max
+    x["k_cache"] = (x["k_cache"].float() * f[None, :, None, None]).to(torch.bfloat16)
+    out, lens, status, _ = run_step(x)
+    assert status == 0
+    assert torch.isfinite(out).all()
+    ref = oracle_step(oracle, x)
+    assert max_err(out, ref) <= TOL[torch.bfloat16]
