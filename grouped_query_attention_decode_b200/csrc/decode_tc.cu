@@ -125,6 +125,43 @@ __device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t bytes) {
     return desc + static_cast<uint64_t>(bytes >> 4);
 }
 
+// Tiles ahead of the copy at which the paged producer loads page ids.
+constexpr int kPageAhead = 2;
+
+// A cursor over the tiles of a CTA's range, one tile at a time, used to look up page ids ahead
+// of the tile being copied.
+struct TileCursor {
+    SegmentWalker w;
+    Segment sg;
+    int jj;
+    bool live;
+
+    __device__ void init(const DecodeParams &p, const CtaRange &cr) {
+        w.init(p, cr);
+        live = w.next(sg);
+        jj = 0;
+    }
+    __device__ void advance() {
+        if (live && ++jj >= sg.len) {
+            live = w.next(sg);
+            jj = 0;
+        }
+    }
+    // Page holding box `box` of the current tile (boxes as the producer cuts them: T / boxr
+    // boxes of min(page_size, T) rows for a full tile, 8-row boxes for a partial one); 0 past
+    // the last box or the last tile.  Every box starts below the sequence's length, so the
+    // block-table index stays below max_pages.
+    __device__ int page_of_box(const DecodeParams &p, int T, int box) const {
+        if (!live) return 0;
+        const int row0 = sg.first + (sg.j0 + jj) * T;
+        const int rows = min(T, sg.n - row0);
+        const int boxr = rows == T ? min(p.page_size, T) : 8;
+        const int nbox = rows == T ? T / boxr : (rows + 7) >> 3;
+        if (box >= nbox) return 0;
+        return __ldg(p.block_table + static_cast<long long>(sg.b) * p.max_pages + (row0 + box * boxr) / p.page_size);
+    }
+};
+
 template <int D, int NH, bool PAGED>
 __global__ void __launch_bounds__(TcCfg<D, NH>::THREADS, 1)
 split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -215,74 +252,87 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     if (warp == 0) {
         // ------------------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            const uint64_t pol = l2_policy_evict_first();
-            SegmentWalker w;
-            w.init(p, cr);
-            Segment sg;
-            int i = 0, sidx = 0;
-            bool ok = true;
-            while (ok && w.next(sg)) {
-                const int qb = sidx % C::QB;
-                if (sidx >= C::QB && !wait_bounded(&sm->q_empty[qb], ((sidx / C::QB) - 1) & 1, abort_flag, budget)) {
-                    ok = false;
-                    break;
-                }
+        // The whole warp walks the tile line; lane 0 waits on the barriers and issues the
+        // copies.  In a paged cache each lane instead owns one box of a tile: it loads that
+        // box's page id kPageAhead tiles ahead of the copy, so the lookup's latency hides behind
+        // the pipeline, and issues the box's copies itself.
+        const uint64_t pol = l2_policy_evict_first();
+        SegmentWalker w;
+        w.init(p, cr);
+        Segment sg;
+        int i = 0, sidx = 0;
+        bool ok = true;
+        [[maybe_unused]] TileCursor ahead;
+        [[maybe_unused]] int pg_ring[kPageAhead];
+        if constexpr (PAGED) {
+            ahead.init(p, cr);
+#pragma unroll
+            for (int k = 0; k < kPageAhead; ++k) {
+                pg_ring[k] = ahead.page_of_box(p, T, lane);
+                ahead.advance();
+            }
+        }
+        while (ok && w.next(sg)) {
+            const int qb = sidx % C::QB;
+            bool got = true;
+            if (lane == 0 && sidx >= C::QB)
+                got = wait_bounded(&sm->q_empty[qb], ((sidx / C::QB) - 1) & 1, abort_flag, budget);
+            if (!__shfl_sync(kFullMask, got, 0)) {
+                ok = false;
+                break;
+            }
+            if (lane == 0) {
                 // q of the unit: rows (token j, head h') of q viewed as (d, H_q, B*Q)
                 mbar_arrive_expect_tx(&sm->q_full[qb], p.q_box_bytes);
 #pragma unroll
                 for (int kb = 0; kb < C::KB; ++kb)
                     tma_load_3d(q_base + qb * C::Q_BYTES + kb * RP * 128, &tm_q, &sm->q_full[qb],
                                 kb * 64, sg.kvh * p.r + sg.hb * p.rb, sg.b * p.Q);
-                ++sidx;
-                for (int jj = 0; jj < sg.len; ++jj) {
-                    const int st = i % S;
-                    const int row0 = sg.first + (sg.j0 + jj) * T;
-                    const int rows = min(T, sg.n - row0);
-                    // Paged cache: page of each box of the tile (boxes of min(page_size, T) rows,
-                    // or 8 rows for a partial tile), loaded before the wait for a free stage so
-                    // that the lookups overlap it.
-                    int page[16];
-                    int boxr = T;
-                    if constexpr (PAGED) {
-                        boxr = rows == T ? min(p.page_size, T) : 8;
-                        const int nbox = rows == T ? T / boxr : (rows + 7) >> 3;
-                        const int32_t *bt = p.block_table + static_cast<long long>(sg.b) * p.max_pages;
+            }
+            ++sidx;
+            for (int jj = 0; jj < sg.len; ++jj) {
+                const int st = i % S;
+                const int row0 = sg.first + (sg.j0 + jj) * T;
+                const int rows = min(T, sg.n - row0);
+                [[maybe_unused]] int pg = 0;
+                if constexpr (PAGED) {
+                    pg = pg_ring[0];
 #pragma unroll
-                        for (int x = 0; x < 16; ++x) {
-                            if (x < nbox) {
-                                int pg = bt[(row0 + x * boxr) / p.page_size];
-                                if (pg < 0 || pg >= p.n_pages) {
-                                    if (p.status != nullptr) atomicOr(p.status, GQA_STATUS_PAGE_RANGE);
-                                    pg = 0;
-                                }
-                                page[x] = pg;
-                            }
+                    for (int k = 0; k + 1 < kPageAhead; ++k) pg_ring[k] = pg_ring[k + 1];
+                    pg_ring[kPageAhead - 1] = ahead.page_of_box(p, T, lane);
+                    ahead.advance();
+                }
+                got = true;
+                if (lane == 0 && i >= S)
+                    got = wait_bounded(&sm->kv_empty[st], ((i / S) - 1) & 1, abort_flag, budget);
+                if (!__shfl_sync(kFullMask, got, 0)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t *kdst = st_base + st * C::STAGE_BYTES;
+                uint8_t *vdst = kdst + C::TILE_BYTES;
+                if constexpr (PAGED) {
+                    // boxes of min(page_size, T) rows, or 8 rows for a partial tile
+                    const int boxr = rows == T ? min(p.page_size, T) : 8;
+                    const int nbox = rows == T ? T / boxr : (rows + 7) >> 3;
+                    if (lane == 0) mbar_arrive_expect_tx(&sm->kv_full[st], 2 * C::KB * nbox * boxr * 128);
+                    __syncwarp();
+                    if (lane < nbox) {
+                        if (pg < 0 || pg >= p.n_pages) {
+                            if (p.status != nullptr) atomicOr(p.status, GQA_STATUS_PAGE_RANGE);
+                            pg = 0;
                         }
-                    }
-                    if (i >= S && !wait_bounded(&sm->kv_empty[st], ((i / S) - 1) & 1, abort_flag, budget)) {
-                        ok = false;
-                        break;
-                    }
-                    uint8_t *kdst = st_base + st * C::STAGE_BYTES;
-                    uint8_t *vdst = kdst + C::TILE_BYTES;
-                    if constexpr (PAGED) {
-                        const int nbox = rows == T ? T / boxr : (rows + 7) >> 3;
                         const CUtensorMap *mk = rows == T ? &tm_k : &tm_k8;
                         const CUtensorMap *mv = rows == T ? &tm_v : &tm_v8;
-                        mbar_arrive_expect_tx(&sm->kv_full[st], 2 * C::KB * nbox * boxr * 128);
+                        const int pr = (row0 + lane * boxr) % p.page_size;
 #pragma unroll
-                        for (int x = 0; x < 16; ++x) {
-                            if (x < nbox) {
-                                const int pr = (row0 + x * boxr) % p.page_size;
-#pragma unroll
-                                for (int kb = 0; kb < C::KB; ++kb) {
-                                    tma_load_4d(kdst + kb * T * 128 + x * boxr * 128, mk, &sm->kv_full[st], kb * 64, sg.kvh, pr, page[x], pol);
-                                    tma_load_4d(vdst + kb * T * 128 + x * boxr * 128, mv, &sm->kv_full[st], kb * 64, sg.kvh, pr, page[x], pol);
-                                }
-                            }
+                        for (int kb = 0; kb < C::KB; ++kb) {
+                            tma_load_4d(kdst + kb * T * 128 + lane * boxr * 128, mk, &sm->kv_full[st], kb * 64, sg.kvh, pr, pg, pol);
+                            tma_load_4d(vdst + kb * T * 128 + lane * boxr * 128, mv, &sm->kv_full[st], kb * 64, sg.kvh, pr, pg, pol);
                         }
-                    } else if (rows == T) {
+                    }
+                } else if (lane == 0) {
+                    if (rows == T) {
                         mbar_arrive_expect_tx(&sm->kv_full[st], C::STAGE_BYTES);
 #pragma unroll
                         for (int kb = 0; kb < C::KB; ++kb) {
@@ -300,9 +350,11 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                             }
                         }
                     }
-                    ++i;
                 }
+                ++i;
             }
+        }
+        if (lane == 0) {
             if (!ok) fail();
             // Drain: no copy may still be writing this CTA's shared memory when it exits.
             for (int ii = (i > S ? i - S : 0); ii < i; ++ii)
