@@ -69,6 +69,20 @@ class Oracle:
         self.lib.oracle_gqa_decode_multi.argtypes = [dp, dp, dp, ip, c_int, c_int, c_int, c_int,
                                                      c_int, c_int, ctypes.c_double, dp, c_int, ip]
         self.lib.oracle_gqa_decode_multi.restype = c_int
+        u8p = ctypes.POINTER(ctypes.c_uint8)
+        fp = ctypes.POINTER(ctypes.c_float)
+        self.lib.oracle_e4m3_value.argtypes = [c_int]
+        self.lib.oracle_e4m3_value.restype = ctypes.c_double
+        self.lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+        self.lib.oracle_e4m3_encode.restype = c_int
+        self.lib.oracle_e4m3_values.argtypes = [u8p, ctypes.c_size_t, dp]
+        self.lib.oracle_e4m3_values.restype = None
+        self.lib.oracle_e4m3_encode_array.argtypes = [fp, ctypes.c_size_t, u8p]
+        self.lib.oracle_e4m3_encode_array.restype = None
+        self.lib.oracle_quantize_rows.argtypes = [dp, ctypes.c_size_t, c_int, c_int, fp, u8p]
+        self.lib.oracle_quantize_rows.restype = None
+        self.lib.oracle_dequantize_rows.argtypes = [u8p, ctypes.c_size_t, c_int, c_int, fp, dp]
+        self.lib.oracle_dequantize_rows.restype = None
         self.lib.oracle_max_threads.argtypes = []
         self.lib.oracle_max_threads.restype = c_int
 
@@ -206,6 +220,94 @@ class Oracle:
         kc, st1 = self.paged_gather(k_pool, block_table, seq_lens)
         vc, st2 = self.paged_gather(v_pool, block_table, seq_lens)
         return self.decode(q, kc, vc, seq_lens, scale)
+
+    # ------------------------------------------------------------------ FP8 (e4m3) cache
+    @staticmethod
+    def _u8(a) -> np.ndarray:
+        return np.ascontiguousarray(a, dtype=np.uint8)
+
+    @staticmethod
+    def _f32(a) -> np.ndarray:
+        return np.ascontiguousarray(a, dtype=np.float32)
+
+    def e4m3_values(self, codes):
+        """float64 value of every e4m3 code (NaN for 0x7F / 0xFF)."""
+        c = self._u8(codes)
+        out = np.empty(c.shape, dtype=np.float64)
+        self.lib.oracle_e4m3_values(c.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)), c.size,
+                                    self._dp(out))
+        return out
+
+    def e4m3_encode(self, x):
+        """Nearest finite e4m3 code of every float32 in x (ties to even, saturating)."""
+        xf = self._f32(x)
+        out = np.empty(xf.shape, dtype=np.uint8)
+        self.lib.oracle_e4m3_encode_array(xf.ctypes.data_as(ctypes.POINTER(ctypes.c_float)),
+                                          xf.size, out.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)))
+        return out
+
+    def quantize(self, x, scale):
+        """Codes of x [..., H_kv, d] (float32 values) with per-head scales [H_kv]."""
+        xd = self._f64(x)
+        sc = self._f32(scale)
+        H_kv, d = xd.shape[-2:]
+        assert sc.shape == (H_kv,)
+        out = np.empty(xd.shape, dtype=np.uint8)
+        self.lib.oracle_quantize_rows(self._dp(xd), xd.size // (H_kv * d), H_kv, d,
+                                      sc.ctypes.data_as(ctypes.POINTER(ctypes.c_float)),
+                                      out.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)))
+        return out
+
+    def dequantize(self, codes, scale):
+        """float64 values value(code) * scale[g] of codes [..., H_kv, d]."""
+        c = self._u8(codes)
+        sc = self._f32(scale)
+        H_kv, d = c.shape[-2:]
+        assert sc.shape == (H_kv,)
+        out = np.empty(c.shape, dtype=np.float64)
+        self.lib.oracle_dequantize_rows(c.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)),
+                                        c.size // (H_kv * d), H_kv, d,
+                                        sc.ctypes.data_as(ctypes.POINTER(ctypes.c_float)), self._dp(out))
+        return out
+
+    def kv_append_fp8(self, k_new, v_new, k_codes, v_codes, k_scale, v_scale, seq_lens):
+        """Quantise the new rows and append them to uint8 code caches [B, L_max, H_kv, d]
+        (in place, with seq_lens).  Returns the status bits."""
+        assert k_codes.dtype == np.uint8 and v_codes.dtype == np.uint8
+        kq = self.quantize(k_new, k_scale).astype(np.float64)
+        vq = self.quantize(v_new, v_scale).astype(np.float64)
+        kc = k_codes.astype(np.float64)
+        vc = v_codes.astype(np.float64)
+        st = self.kv_append(kq, vq, kc, vc, seq_lens)
+        k_codes[...] = kc.astype(np.uint8)
+        v_codes[...] = vc.astype(np.uint8)
+        return st
+
+    def kv_append_paged_fp8(self, k_new, v_new, k_pool, v_pool, k_scale, v_scale, block_table,
+                            seq_lens):
+        """Paged form of kv_append_fp8 on uint8 code pools [n_pages, page_size, H_kv, d]."""
+        assert k_pool.dtype == np.uint8 and v_pool.dtype == np.uint8
+        kq = self.quantize(k_new, k_scale).astype(np.float64)
+        vq = self.quantize(v_new, v_scale).astype(np.float64)
+        kp = k_pool.astype(np.float64)
+        vp = v_pool.astype(np.float64)
+        st = self.kv_append_paged(kq, vq, kp, vp, block_table, seq_lens)
+        k_pool[...] = kp.astype(np.uint8)
+        v_pool[...] = vp.astype(np.uint8)
+        return st
+
+    def decode_fp8(self, q, k_codes, v_codes, k_scale, v_scale, seq_lens, scale: float,
+                   window: int = 0, nthreads: int = 0):
+        """Decode over an e4m3 cache: the oracle decode on the dequantised values."""
+        kc = self.dequantize(k_codes, k_scale)
+        vc = self.dequantize(v_codes, v_scale)
+        return self.decode_window(q, kc, vc, seq_lens, window, scale, nthreads=nthreads)
+
+    def decode_paged_fp8(self, q, k_pool, v_pool, k_scale, v_scale, block_table, seq_lens,
+                         scale: float):
+        """Paged decode over e4m3 pools: dequantise the pools, gather, decode."""
+        return self.decode_paged(q, self.dequantize(k_pool, k_scale),
+                                 self.dequantize(v_pool, v_scale), block_table, seq_lens, scale)
 
 
 _default: Oracle | None = None

@@ -275,6 +275,81 @@ void oracle_kv_append_paged(const double *k_new, const double *v_new, double *k_
     }
 }
 
+/* ---------------------------------------------------------------------- FP8 (e4m3) cache
+ * "GQA 阅读笔记", section "复现性与工程实践", item "混合精度": serving systems keep the KV cache
+ * in FP8, and that halves the per-step KV bytes again on top of GQA's saving.  Page 3 (the
+ * FlashAttention-2 GQA article), section 4.2 item 3: the cache may be stored in FP8 and
+ * dequantised when read.  Neither page fixes the format or the scaling.  Reading taken here:
+ * the OCP FP8 E4M3 format (1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits; no
+ * infinities; exponent 1111 with mantissa 111 is NaN; largest finite magnitude 448), one
+ * float32 scale per key/value head for K and another for V, and a stored code c of head g
+ * standing for value(c) * scale[g].  Quantising x takes the code nearest to the float32
+ * quotient x / scale[g] (float32 division), ties to the code with an even mantissa, and
+ * magnitudes past 448 to +-448 (saturation); NaN becomes 0x7F.
+ *
+ * Appends and page gathers of codes reuse the float64 routines above: a code 0..255 held in a
+ * double moves through them unchanged. */
+
+/* The value a code stands for, from the field definitions. */
+double oracle_e4m3_value(int code) {
+    int sign = (code >> 7) & 1, e = (code >> 3) & 15, m = code & 7;
+    if (e == 15 && m == 7) return NAN;
+    double mag = e == 0 ? ldexp(m / 8.0, -6) : ldexp(1.0 + m / 8.0, e - 7);
+    return sign ? -mag : mag;
+}
+
+/* The code nearest to x among the finite ones, by brute force over all 127 non-negative finite
+ * codes: the smallest distance wins, a tie goes to the code with an even mantissa (its lowest
+ * bit clear).  Past 448 the nearest finite code is 448 itself, which is the saturation. */
+int oracle_e4m3_encode(float x) {
+    if (isnan(x)) return 0x7F;
+    double a = fabs((double)x);
+    /* every finite code is at most 448, so from 448 up the nearest one is 448 itself (the
+     * distances of a huge x would also round to equal values) */
+    if (a >= 448.0) return signbit(x) ? 0xFE : 0x7E;
+    int best = 0;
+    double best_dist = INFINITY;
+    for (int c = 0; c < 127; ++c) {
+        double dist = fabs(oracle_e4m3_value(c) - a);
+        if (dist < best_dist || (dist == best_dist && (c & 1) == 0 && (best & 1) == 1)) {
+            best = c;
+            best_dist = dist;
+        }
+    }
+    return signbit(x) ? (best | 0x80) : best;
+}
+
+void oracle_e4m3_values(const uint8_t *codes, size_t n, double *out) {
+    for (size_t i = 0; i < n; ++i) out[i] = oracle_e4m3_value(codes[i]);
+}
+
+void oracle_e4m3_encode_array(const float *x, size_t n, uint8_t *codes) {
+    for (size_t i = 0; i < n; ++i) codes[i] = (uint8_t)oracle_e4m3_encode(x[i]);
+}
+
+/* Rows of [n_rows][H_kv][d] values (each exactly a float32) to codes with per-head scales. */
+void oracle_quantize_rows(const double *x, size_t n_rows, int H_kv, int d, const float *scale,
+                          uint8_t *codes) {
+    for (size_t r = 0; r < n_rows; ++r)
+        for (int g = 0; g < H_kv; ++g)
+            for (int i = 0; i < d; ++i) {
+                size_t at = (r * H_kv + g) * d + i;
+                float quotient = (float)x[at] / scale[g];
+                codes[at] = (uint8_t)oracle_e4m3_encode(quotient);
+            }
+}
+
+/* Codes of [n_rows][H_kv][d] back to values: value(code) * scale[g], exact in float64. */
+void oracle_dequantize_rows(const uint8_t *codes, size_t n_rows, int H_kv, int d,
+                            const float *scale, double *out) {
+    for (size_t r = 0; r < n_rows; ++r)
+        for (int g = 0; g < H_kv; ++g)
+            for (int i = 0; i < d; ++i) {
+                size_t at = (r * H_kv + g) * d + i;
+                out[at] = oracle_e4m3_value(codes[at]) * (double)scale[g];
+            }
+}
+
 /* Number of threads the OpenMP runtime will use for the next parallel region. */
 int oracle_max_threads(void) {
 #ifdef _OPENMP

@@ -378,12 +378,110 @@ def pin_multi_query(o):
     assert st & 2  # fewer rows than query tokens
 
 
+def _torch_e4m3_values(codes):
+    """torch's float8_e4m3fn reading of uint8 codes, as float64."""
+    return torch.from_numpy(np.ascontiguousarray(codes, dtype=np.uint8)).view(torch.float8_e4m3fn).double().numpy()
+
+
+def _torch_e4m3_encode(x):
+    """torch's round-to-nearest-even float32 -> float8_e4m3fn (inputs within +-448)."""
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def pin_fp8_codec(o):
+    """The e4m3 codec ("GQA 阅读笔记", section "复现性与工程实践", mixed precision: an FP8 KV
+    cache): every code reads as torch's float8_e4m3fn does; closed-form values of the format
+    (1, 448, the smallest normal and subnormal, NaN); codes round-trip; encoding agrees with
+    torch's round-to-nearest-even on random values and on every midpoint between neighbouring
+    codes (ties go to the even mantissa); magnitudes past 448 and infinities saturate; the
+    rounding error stays within half a unit in the last place."""
+    codes = np.arange(256, dtype=np.uint8)
+    v = o.e4m3_values(codes)
+    t = _torch_e4m3_values(codes)
+    assert np.array_equal(np.isnan(v), np.isnan(t))
+    fin = ~np.isnan(v)
+    assert np.array_equal(v[fin], t[fin])
+    assert np.array_equal(np.signbit(v[fin]), np.signbit(t[fin]))
+    assert np.isnan(v[0x7F]) and np.isnan(v[0xFF]) and int(np.isnan(v).sum()) == 2
+    assert v[0x38] == 1.0 and v[0x7E] == 448.0 and v[0xFE] == -448.0
+    assert v[0x08] == 2.0 ** -6 and v[0x01] == 2.0 ** -9 and v[0x07] == 7 * 2.0 ** -9
+    assert v[0x00] == 0.0 and np.signbit(v[0x80])
+    # round trip of every finite code
+    finite_codes = codes[fin]
+    assert np.array_equal(o.e4m3_encode(v[fin].astype(np.float32)), finite_codes)
+    # midpoints between neighbouring positive codes: the even mantissa wins
+    pos = v[:127]
+    mids = ((pos[:-1] + pos[1:]) / 2).astype(np.float32)
+    assert np.array_equal(mids.astype(np.float64), (pos[:-1] + pos[1:]) / 2)  # exact in float32
+    enc = o.e4m3_encode(mids)
+    want = np.where(np.arange(126) % 2 == 0, np.arange(126), np.arange(1, 127)).astype(np.uint8)
+    assert np.array_equal(enc, want)
+    assert np.array_equal(enc, _torch_e4m3_encode(mids))
+    assert np.array_equal(o.e4m3_encode(-mids), want | 0x80)
+    r = _rng(303)
+    x = np.concatenate([r.standard_normal(20000) * 40, r.standard_normal(20000) * 0.01,
+                        r.uniform(-448, 448, 20000)]).astype(np.float32)
+    assert np.array_equal(o.e4m3_encode(x), _torch_e4m3_encode(x))
+    # saturation
+    sat = np.array([448.0, 449.0, 463.9, 464.0, 500.0, 1e30, np.inf], dtype=np.float32)
+    assert np.all(o.e4m3_encode(sat) == 0x7E) and np.all(o.e4m3_encode(-sat) == 0xFE)
+    assert o.e4m3_encode(np.array([np.nan], dtype=np.float32))[0] == 0x7F
+    # half-ulp bound: 2^-4 relative on normals, 2^-10 absolute below 2^-6
+    y = o.e4m3_values(o.e4m3_encode(x)).astype(np.float64)
+    err = np.abs(y - x.astype(np.float64))
+    normal = np.abs(x) >= 2.0 ** -6
+    assert np.all(err[normal] <= 2.0 ** -4 * np.abs(x[normal].astype(np.float64)))
+    assert np.all(err[~normal] <= 2.0 ** -10)
+
+
+def pin_fp8_cache(o):
+    """The FP8 cache with one scale per key/value head: quantising divides by the head's scale
+    in float32 and rounds as torch does; dequantising multiplies back exactly; the append puts
+    the quantised rows at row seq_lens[b] and refuses a full cache; the decode over codes equals
+    torch's fp64 SDPA over the dequantised values (dequantised by torch)."""
+    r = _rng(404)
+    B, H_q, H_kv, d, L = 3, 8, 2, 32, 40
+    k_scale = (r.uniform(0.5, 2.0, H_kv) / 64).astype(np.float32)
+    v_scale = (r.uniform(0.5, 2.0, H_kv) / 64).astype(np.float32)
+    x = r.standard_normal((5, H_kv, d)).astype(np.float32)
+    codes = o.quantize(x, k_scale)
+    want = _torch_e4m3_encode(np.clip(x / k_scale[None, :, None], -448, 448))
+    assert np.array_equal(codes, want)
+    deq = o.dequantize(codes, k_scale)
+    assert np.array_equal(deq, _torch_e4m3_values(codes) * k_scale.astype(np.float64)[None, :, None])
+    # append: codes of the new rows land at row seq_lens[b]
+    k_codes = o.quantize(r.standard_normal((B, L, H_kv, d)).astype(np.float32), k_scale)
+    v_codes = o.quantize(r.standard_normal((B, L, H_kv, d)).astype(np.float32), v_scale)
+    lens = np.array([0, 17, L], dtype=np.int32)
+    kn = r.standard_normal((B, H_kv, d)).astype(np.float32)
+    vn = r.standard_normal((B, H_kv, d)).astype(np.float32)
+    kc2, vc2, l2 = k_codes.copy(), v_codes.copy(), lens.copy()
+    st = o.kv_append_fp8(kn, vn, kc2, vc2, k_scale, v_scale, l2)
+    assert st == 1 and list(l2) == [1, 18, L]
+    for b, t in ((0, 0), (1, 17)):
+        assert np.array_equal(kc2[b, t], o.quantize(kn[b][None], k_scale)[0])
+        assert np.array_equal(vc2[b, t], o.quantize(vn[b][None], v_scale)[0])
+        mask = np.ones(L, dtype=bool)
+        mask[t] = False
+        assert np.array_equal(kc2[b, mask], k_codes[b, mask])
+    assert np.array_equal(kc2[2], k_codes[2])
+    # decode over codes == SDPA over torch-dequantised values
+    q = r.standard_normal((B, H_q, d))
+    lens = np.array([40, 1, 23], dtype=np.int32)
+    Kd = _torch_e4m3_values(k_codes) * k_scale.astype(np.float64)[None, None, :, None]
+    Vd = _torch_e4m3_values(v_codes) * v_scale.astype(np.float64)[None, None, :, None]
+    got = o.decode_fp8(q, k_codes, v_codes, k_scale, v_scale, lens, 0.2)
+    assert np.max(np.abs(got - _sdpa_reference(q, Kd, Vd, lens, 0.2))) <= 1e-12
+    got_w = o.decode_fp8(q, k_codes, v_codes, k_scale, v_scale, lens, 0.2, window=7)
+    assert np.array_equal(got_w, o.decode_window(q, Kd, Vd, lens, 7, 0.2))
+
+
 ALL_PINS = [
     pin_append_position, pin_append_overflow, pin_expand_matches_repeat_interleave,
     pin_single_head_vs_sdpa, pin_decode_vs_sdpa_gqa, pin_mha_endpoint, pin_mqa_endpoint,
     pin_expand_then_attend_equivalence, pin_grouping_changes_output, pin_closed_forms,
     pin_invariants, pin_brute_force_tiny, pin_empty_and_range, pin_divisibility, pin_window,
-    pin_paged, pin_multi_query,
+    pin_paged, pin_multi_query, pin_fp8_codec, pin_fp8_cache,
 ]
 
 

@@ -40,3 +40,12 @@ def test_cache_shrinks_with_kv_heads_and_multiplies_do_not():
         assert counts.decode_step_multiplies(lens, 64, 128) == base_mults
     full = counts.attention_multiplies_full_pass(8, 10, 4)
     assert full == {"scores": 3200, "weighted_sum": 3200}
+
+
+@pytest.mark.parametrize("row", _rows("kv_bytes_ratios.txt"), ids=lambda r: r[0])
+def test_printed_fp8_bandwidth_ratios(row):
+    _, h_a, b_a, h_b, b_b, expected, _cite = row
+    for B, N, L, d in ((1, 1, 1, 128), (16, 80, 4096, 128), (3, 2, 17, 64)):
+        a = counts.kv_cache_bytes(B, N, L, int(h_a), d, int(b_a))
+        b = counts.kv_cache_bytes(B, N, L, int(h_b), d, int(b_b))
+        assert a == int(expected) * b

@@ -43,6 +43,15 @@ MUTANTS = {
     "multi_off_by_one": ("int rows = n - Q + 1 + j;", "int rows = n - Q + j;"),
     "window_off_by_one": ("int first = (window > 0 && n > window) ? n - window : 0;",
                           "int first = (window > 0 && n > window) ? n - window + 1 : 0;"),
+    "e4m3_exponent_bias": ("ldexp(1.0 + m / 8.0, e - 7)", "ldexp(1.0 + m / 8.0, e - 8)"),
+    "e4m3_subnormal_scale": ("ldexp(m / 8.0, -6)", "ldexp(m / 8.0, -7)"),
+    "e4m3_ties_down": ("(dist == best_dist && (c & 1) == 0 && (best & 1) == 1)", "0"),
+    "e4m3_no_saturation": ("if (a >= 448.0) return signbit(x) ? 0xFE : 0x7E;",
+                           "if (a >= 448.0) return 0x7F;"),
+    "quantize_multiplies": ("float quotient = (float)x[at] / scale[g];",
+                            "float quotient = (float)x[at] * scale[g];"),
+    "dequantize_first_head_scale": ("out[at] = oracle_e4m3_value(codes[at]) * (double)scale[g];",
+                                    "out[at] = oracle_e4m3_value(codes[at]) * (double)scale[0];"),
 }
 
 
