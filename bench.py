@@ -187,12 +187,26 @@ def bench_ours(args, rank, world, local):
         nws = gqa.load_library().gqa_decode_multi_workspace_size(w.B, w.queries, w.H_q, w.H_kv, w.d,
                                                                  gqa.DTYPE_BF16 if w.dtype == torch.bfloat16 else gqa.DTYPE_F32)
         ws = torch.empty(nws, dtype=torch.uint8, device=dev)
+    elif w.fp8:
+        ws = gqa.alloc_workspace_fp8(w.B, w.H_q, w.H_kv, w.d, device=dev)
     else:
         ws = gqa.alloc_workspace(w.B, w.H_q, w.H_kv, w.d, w.dtype, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
+    ks = x["k_scale"].to(dev) if w.fp8 else None
+    vs = x["v_scale"].to(dev) if w.fp8 else None
 
     def step(i, lens_row, qq=q, kk=kn, vv=vn):
         kc, vc = caches[i & 1]
+        if w.fp8:
+            if block_table is not None:
+                gqa.kv_append_paged_fp8(kk, vv, kc, vc, ks, vs, block_table, lens_row, status=status)
+                gqa.decode_paged_fp8(qq, kc, vc, ks, vs, block_table, lens_row, x["scale"], out=out,
+                                     workspace=ws, status=status)
+            else:
+                gqa.kv_append_fp8(kk, vv, kc, vc, ks, vs, lens_row, status=status)
+                gqa.decode_fp8(qq, kc, vc, ks, vs, lens_row, x["scale"], window=w.window, out=out,
+                               workspace=ws, status=status)
+            return
         if block_table is not None:
             gqa.kv_append_paged(kk, vv, kc, vc, block_table, lens_row, status=status)
             gqa.decode_paged(qq, kc, vc, block_table, lens_row, x["scale"], out=out, workspace=ws,
@@ -331,7 +345,7 @@ def bench_ours(args, rank, world, local):
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
-            "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32",
+            "dtype": "e4m3" if w.fp8 else ("bf16" if w.dtype == torch.bfloat16 else "f32"),
             "data": "synthetic",
             "config": {
                 "workload": w.name, "B": w.B, "H_q": w.H_q, "H_kv": w.H_kv, "d": w.d,
@@ -339,7 +353,8 @@ def bench_ours(args, rank, world, local):
                 "window": w.window or None,
                 "page_size": w.page_size or None,
                 "query_tokens": w.queries,
-                "sum_seq_lens": int(sum(lengths)), "kv_dtype": str(w.dtype).replace("torch.", ""),
+                "sum_seq_lens": int(sum(lengths)),
+                "kv_dtype": "e4m3 (per-head scales)" if w.fp8 else str(w.dtype).replace("torch.", ""),
                 "accumulate": "f32", "ideal_kv_bytes_per_step": ideal,
                 "parallelism": f"replicas x{world}",
                 "l2": "inputs larger than L2: two cache copies alternate between steps "
@@ -347,7 +362,8 @@ def bench_ours(args, rank, world, local):
             },
             "gpu_launches": 3 * K,
             "roofline": {
-                "bound": "hbm", "kernel": "split_tc_kernel", "achieved": round(achieved, 1),
+                "bound": "hbm", "kernel": "split_tc8_kernel" if w.fp8 else "split_tc_kernel",
+                "achieved": round(achieved, 1),
                 "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                 "frac": round(achieved / peak, 4),
                 "traffic": profiled_traffic(w.name),
@@ -386,11 +402,19 @@ def cpu_baseline(w, x, budget_s, steps=None):
         xb = {k: (v[b:b + 1] if isinstance(v, torch.Tensor) and v.dim() > 0 and v.shape[0] == B else v)
               for k, v in x.items()}
         q = xb["q"].double().numpy()
-        kc = xb["k_cache"].double().numpy().copy()
-        vc = xb["v_cache"].double().numpy().copy()
         lens = xb["seq_lens_pre"].numpy().copy()
+        if w.fp8:
+            kc = xb["k_cache"].numpy().copy()
+            vc = xb["v_cache"].numpy().copy()
+            ksc, vsc = x["k_scale"].numpy(), x["v_scale"].numpy()
+        else:
+            kc = xb["k_cache"].double().numpy().copy()
+            vc = xb["v_cache"].double().numpy().copy()
         ts = time.perf_counter()
-        if w.queries > 1:
+        if w.fp8:
+            o.kv_append_fp8(xb["k_new"].float().numpy(), xb["v_new"].float().numpy(), kc, vc, ksc, vsc, lens)
+            o.decode_fp8(q, kc, vc, ksc, vsc, lens, x["scale"], window=w.window)
+        elif w.queries > 1:
             for j in range(w.queries):  # the Q drafted rows, in order
                 o.kv_append(xb["k_new"][:, j].double().numpy(), xb["v_new"][:, j].double().numpy(), kc, vc, lens)
             o.decode_multi(q, kc, vc, lens, x["scale"])
@@ -431,9 +455,23 @@ def profile_run(args, local):
         block_table = paged["block_table"].to(dev)
     lens_rows = x["seq_lens_pre"].to(dev).repeat(args.warmup + args.steps, 1).contiguous()
     out = torch.empty((w.B, w.H_q, w.d), dtype=torch.float32, device=dev)
-    ws = gqa.alloc_workspace(w.B, w.H_q, w.H_kv, w.d, w.dtype, device=dev)
+    if w.fp8:
+        ws = gqa.alloc_workspace_fp8(w.B, w.H_q, w.H_kv, w.d, device=dev)
+        ks, vs = x["k_scale"].to(dev), x["v_scale"].to(dev)
+    else:
+        ws = gqa.alloc_workspace(w.B, w.H_q, w.H_kv, w.d, w.dtype, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     for i in range(args.warmup + args.steps):
+        if w.fp8:
+            if block_table is not None:
+                gqa.kv_append_paged_fp8(kn, vn, kc, vc, ks, vs, block_table, lens_rows[i], status=status)
+                gqa.decode_paged_fp8(q, kc, vc, ks, vs, block_table, lens_rows[i], x["scale"], out=out,
+                                     workspace=ws, status=status)
+            else:
+                gqa.kv_append_fp8(kn, vn, kc, vc, ks, vs, lens_rows[i], status=status)
+                gqa.decode_fp8(q, kc, vc, ks, vs, lens_rows[i], x["scale"], window=w.window, out=out,
+                               workspace=ws, status=status)
+            continue
         if block_table is not None:
             gqa.kv_append_paged(kn, vn, kc, vc, block_table, lens_rows[i], status=status)
             gqa.decode_paged(q, kc, vc, block_table, lens_rows[i], x["scale"], out=out,

@@ -31,7 +31,9 @@ STATUS_PAGE_RANGE = 16
 EXPORTED = ("gqa_kv_append", "gqa_decode_workspace_size", "gqa_decode", "gqa_status_string",
             "gqa_set_wait_timeout_ns", "gqa_profile_events", "gqa_decode_noalloc",
             "gqa_decode_window", "gqa_kv_append_paged", "gqa_decode_paged",
-            "gqa_kv_append_multi", "gqa_decode_multi_workspace_size", "gqa_decode_multi")
+            "gqa_kv_append_multi", "gqa_decode_multi_workspace_size", "gqa_decode_multi",
+            "gqa_kv_append_fp8", "gqa_kv_append_paged_fp8", "gqa_decode_fp8",
+            "gqa_decode_paged_fp8")
 
 
 class GQAError(RuntimeError):
@@ -83,6 +85,20 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gqa_decode_noalloc.argtypes = [vp, vp, vp, i32p, c_int, c_int, c_int, c_int, c_int,
                                        ctypes.c_float, c_int, vp, i32p, vp]
     lib.gqa_decode_noalloc.restype = c_int
+    fp = ctypes.POINTER(ctypes.c_float)
+    lib.gqa_kv_append_fp8.argtypes = [vp, vp, c_int, vp, vp, vp, vp, i32p, c_int, c_int, c_int,
+                                      c_int, i32p, vp]
+    lib.gqa_kv_append_fp8.restype = c_int
+    lib.gqa_kv_append_paged_fp8.argtypes = [vp, vp, c_int, vp, vp, vp, vp, i32p, c_int, i32p,
+                                            c_int, c_int, c_int, c_int, c_int, i32p, vp]
+    lib.gqa_kv_append_paged_fp8.restype = c_int
+    lib.gqa_decode_fp8.argtypes = [vp, vp, vp, vp, vp, i32p, c_int, c_int, c_int, c_int, c_int,
+                                   c_int, ctypes.c_float, vp, vp, ctypes.c_size_t, i32p, vp]
+    lib.gqa_decode_fp8.restype = c_int
+    lib.gqa_decode_paged_fp8.argtypes = [vp, vp, vp, vp, vp, i32p, c_int, i32p, c_int, c_int,
+                                         c_int, c_int, c_int, c_int, ctypes.c_float, vp, vp,
+                                         ctypes.c_size_t, i32p, vp]
+    lib.gqa_decode_paged_fp8.restype = c_int
     lib.gqa_status_string.argtypes = [c_int]
     lib.gqa_status_string.restype = ctypes.c_char_p
     lib.gqa_set_wait_timeout_ns.argtypes = [ctypes.c_ulonglong]
@@ -255,3 +271,94 @@ def profile_events(before_split=None, after_split=None) -> None:
     a = ctypes.c_void_p(before_split.cuda_event) if before_split is not None else None
     b = ctypes.c_void_p(after_split.cuda_event) if after_split is not None else None
     _check(load_library().gqa_profile_events(a, b))
+
+
+# ------------------------------------------------------------------ FP8 (e4m3) cache
+DTYPE_E4M3 = 2
+
+
+def _codes(t: torch.Tensor) -> torch.Tensor:
+    """An e4m3 cache as bytes: torch.uint8, or torch.float8_e4m3fn viewed as uint8."""
+    if t.dtype == torch.float8_e4m3fn:
+        return t.view(torch.uint8)
+    if t.dtype != torch.uint8:
+        raise ValueError(f"an e4m3 cache must be uint8 or float8_e4m3fn, not {t.dtype}")
+    return t
+
+
+def _scales(t: torch.Tensor, H_kv: int) -> torch.Tensor:
+    if t.dtype != torch.float32 or t.shape != (H_kv,):
+        raise ValueError(f"scales must be float32 [{H_kv}]")
+    return t
+
+
+def alloc_workspace_fp8(B: int, H_q: int, H_kv: int, d: int, device=None):
+    n = int(load_library().gqa_decode_workspace_size(B, H_q, H_kv, d, DTYPE_E4M3))
+    if n == 0:
+        raise GQAError(-9, "no usable sm_100 device is current, or invalid sizes")
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def kv_append_fp8(k_new, v_new, k_cache, v_cache, k_scale, v_scale, seq_lens, status=None,
+                  stream=None) -> None:
+    """gqa_kv_append_fp8: quantise k_new/v_new [B, H_kv, d] (bf16 or float32) to e4m3 codes of
+    their head's scale and write them at row seq_lens[b]; then seq_lens[b] += 1."""
+    kc, vc = _codes(k_cache), _codes(v_cache)
+    B, L_max, H_kv, d = kc.shape
+    _check(load_library().gqa_kv_append_fp8(
+        _ptr(k_new), _ptr(v_new), _dtype(k_new), _ptr(kc), _ptr(vc),
+        _ptr(_scales(k_scale, H_kv)), _ptr(_scales(v_scale, H_kv)), _ptr(seq_lens), B, H_kv, d,
+        L_max, _ptr(status), _stream(stream)))
+
+
+def kv_append_paged_fp8(k_new, v_new, k_pool, v_pool, k_scale, v_scale, block_table, seq_lens,
+                        status=None, stream=None) -> None:
+    """gqa_kv_append_paged_fp8: the quantising append into e4m3 page pools."""
+    kp, vp_ = _codes(k_pool), _codes(v_pool)
+    n_pages, page_size, H_kv, d = kp.shape
+    B, max_pages = block_table.shape
+    _check(load_library().gqa_kv_append_paged_fp8(
+        _ptr(k_new), _ptr(v_new), _dtype(k_new), _ptr(kp), _ptr(vp_),
+        _ptr(_scales(k_scale, H_kv)), _ptr(_scales(v_scale, H_kv)), _ptr(block_table), max_pages,
+        _ptr(seq_lens), B, H_kv, d, page_size, n_pages, _ptr(status), _stream(stream)))
+
+
+def decode_fp8(q, k_cache, v_cache, k_scale, v_scale, seq_lens, scale: float, window: int = 0,
+               out=None, workspace=None, status=None, stream=None) -> torch.Tensor:
+    """gqa_decode_fp8: the decode over an e4m3 cache (window > 0: sliding window).  q is bf16
+    [B, H_q, d]; returns out [B, H_q, d] float32."""
+    kc, vc = _codes(k_cache), _codes(v_cache)
+    B, H_q, d = q.shape
+    _, L_max, H_kv, _ = kc.shape
+    if q.dtype != torch.bfloat16:
+        raise ValueError("q must be bfloat16 for an e4m3 cache")
+    if out is None:
+        out = torch.empty((B, H_q, d), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace_fp8(B, H_q, H_kv, d, device=q.device)
+    _check(load_library().gqa_decode_fp8(
+        _ptr(q), _ptr(kc), _ptr(vc), _ptr(_scales(k_scale, H_kv)), _ptr(_scales(v_scale, H_kv)),
+        _ptr(seq_lens), B, H_q, H_kv, d, L_max, int(window), float(scale), _ptr(out),
+        _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream)))
+    return out
+
+
+def decode_paged_fp8(q, k_pool, v_pool, k_scale, v_scale, block_table, seq_lens, scale: float,
+                     out=None, workspace=None, status=None, stream=None) -> torch.Tensor:
+    """gqa_decode_paged_fp8: the decode over e4m3 page pools."""
+    kp, vp_ = _codes(k_pool), _codes(v_pool)
+    B, H_q, d = q.shape
+    n_pages, page_size, H_kv, _ = kp.shape
+    _, max_pages = block_table.shape
+    if q.dtype != torch.bfloat16:
+        raise ValueError("q must be bfloat16 for an e4m3 cache")
+    if out is None:
+        out = torch.empty((B, H_q, d), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace_fp8(B, H_q, H_kv, d, device=q.device)
+    _check(load_library().gqa_decode_paged_fp8(
+        _ptr(q), _ptr(kp), _ptr(vp_), _ptr(_scales(k_scale, H_kv)), _ptr(_scales(v_scale, H_kv)),
+        _ptr(block_table), max_pages, _ptr(seq_lens), B, H_q, H_kv, d, page_size, n_pages,
+        float(scale), _ptr(out), _ptr(workspace), workspace.numel(), _ptr(status),
+        _stream(stream)))
+    return out

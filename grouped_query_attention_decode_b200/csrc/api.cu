@@ -71,8 +71,11 @@ Geometry geometry(int B, int H_q, int H_kv, int d, int G, int Q = 1) {
     return g;
 }
 
-int check_shape(int B, int H_q, int H_kv, int d, int L_max, gqa_dtype_t dtype) {
-    if (dtype != GQA_DTYPE_F32 && dtype != GQA_DTYPE_BF16) return GQA_ERR_UNSUPPORTED_DTYPE;
+int check_shape(int B, int H_q, int H_kv, int d, int L_max, gqa_dtype_t dtype,
+                bool allow_e4m3 = false) {
+    if (dtype != GQA_DTYPE_F32 && dtype != GQA_DTYPE_BF16 &&
+        !(allow_e4m3 && dtype == GQA_DTYPE_E4M3))
+        return GQA_ERR_UNSUPPORTED_DTYPE;
     if (B <= 0 || H_q <= 0 || H_kv <= 0 || L_max <= 0) return GQA_ERR_SHAPE;
     if (H_q % H_kv != 0) return GQA_ERR_HEADS_NOT_DIVISIBLE;
     if (d != 64 && d != 128) return GQA_ERR_UNSUPPORTED_DIM;
@@ -114,6 +117,25 @@ bool encode_cache_map(CUtensorMap *m, const void *base, int B, int H_kv, int d, 
     return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims,
                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// An e4m3 cache as (d, H_kv, rows, sequences or pages) of bytes; boxes of `rows` rows of one
+// key/value head, d bytes wide, swizzled as the UMMA operands expect (128-byte swizzle for
+// d = 128, 64-byte for d = 64).
+bool encode_cache_map8(CUtensorMap *m, const void *base, int outer, int H_kv, int d, int rows_dim,
+                       int rows) {
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H_kv),
+                                static_cast<cuuint64_t>(rows_dim), static_cast<cuuint64_t>(outer)};
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(d),
+                                   static_cast<cuuint64_t>(H_kv) * d,
+                                   static_cast<cuuint64_t>(rows_dim) * H_kv * d};
+    const cuuint32_t box[4] = {static_cast<cuuint32_t>(d), 1, static_cast<cuuint32_t>(rows), 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void *>(base), dims,
+                       strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                       d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -185,7 +207,7 @@ extern "C" size_t gqa_decode_multi_workspace_size(int B, int Q, int H_q, int H_k
 }
 
 extern "C" size_t gqa_decode_workspace_size(int B, int H_q, int H_kv, int d, gqa_dtype_t dtype) {
-    if (check_shape(B, H_q, H_kv, d, 1, dtype) != GQA_OK) return 0;
+    if (check_shape(B, H_q, H_kv, d, 1, dtype, true) != GQA_OK) return 0;
     int dev = 0;
     const int sms = current_sm_count(&dev);
     if (sms <= 0) return 0;
@@ -204,10 +226,13 @@ int decode_impl(const void *q, const void *k_cache, const void *v_cache, const i
                 int B, int H_q, int H_kv, int d, int L_max, int window, float scale,
                 gqa_dtype_t dtype, float *out, void *workspace, size_t workspace_bytes,
                 int32_t *status, cudaStream_t stream, const PagedArgs &pg = PagedArgs(),
-                int Q = 1) {
+                int Q = 1, const float *k_scale = nullptr, const float *v_scale = nullptr) {
     if (!q || !k_cache || !v_cache || !seq_lens || !out) return GQA_ERR_NULL;
-    const int rc = check_shape(B, H_q, H_kv, d, L_max, dtype);
+    const bool fp8 = k_scale != nullptr;
+    const int rc = check_shape(B, H_q, H_kv, d, L_max, dtype, fp8);
     if (rc != GQA_OK) return rc;
+    if (fp8 && (dtype != GQA_DTYPE_E4M3 || !v_scale)) return GQA_ERR_NULL;
+    if (fp8 && (!aligned(k_scale, 4) || !aligned(v_scale, 4))) return GQA_ERR_ALIGNMENT;
     if (!workspace) return GQA_ERR_WORKSPACE;
     if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16) ||
         !aligned(seq_lens, 4) || !aligned(workspace, 256) || (status && !aligned(status, 4)))
@@ -237,7 +262,9 @@ int decode_impl(const void *q, const void *k_cache, const void *v_cache, const i
     p.RB = g.RB;
     p.HB = g.HB;
     p.UB = g.UB;
-    p.T = dtype == GQA_DTYPE_BF16 ? 128 : 64;
+    p.T = fp8 ? tc8_tile_rows(g.RB) : (dtype == GQA_DTYPE_BF16 ? 128 : 64);
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
     p.window = window;
     p.block_table = pg.block_table;
     p.max_pages = pg.max_pages;
@@ -256,7 +283,20 @@ int decode_impl(const void *q, const void *k_cache, const void *v_cache, const i
     cudaEvent_t ev0 = g_ev_before.load(), ev1 = g_ev_after.load();
     const bool profile = ev0 != nullptr && ev1 != nullptr;
     int res;
-    if (dtype == GQA_DTYPE_BF16) {
+    if (fp8) {
+        if (encode_fn() == nullptr) return GQA_ERR_CUDA;
+        TmaMaps maps;
+        const int rows_dim = pg.block_table ? pg.page_size : L_max;
+        const int outer_dim = pg.block_table ? pg.n_pages : B;
+        const int box = pg.block_table ? (pg.page_size < p.T ? pg.page_size : p.T) : p.T;
+        if (!encode_cache_map8(&maps.k, k_cache, outer_dim, H_kv, d, rows_dim, box) ||
+            !encode_cache_map8(&maps.k8, k_cache, outer_dim, H_kv, d, rows_dim, 8) ||
+            !encode_cache_map8(&maps.v, v_cache, outer_dim, H_kv, d, rows_dim, box) ||
+            !encode_cache_map8(&maps.v8, v_cache, outer_dim, H_kv, d, rows_dim, 8))
+            return GQA_ERR_SHAPE;
+        if (profile && cudaEventRecord(ev0, stream) != cudaSuccess) return GQA_ERR_CUDA;
+        res = launch_split_tc8(maps, q, p, stream);
+    } else if (dtype == GQA_DTYPE_BF16) {
         const int rp = tc_q_box_rows(g.RB);
         if (encode_fn() == nullptr) return GQA_ERR_CUDA;
         TmaMaps maps;
@@ -356,6 +396,88 @@ extern "C" int gqa_decode_window(const void *q, const void *k_cache, const void 
     if (window <= 0) return GQA_ERR_SHAPE;
     return decode_impl(q, k_cache, v_cache, seq_lens, B, H_q, H_kv, d, L_max, window, scale,
                        dtype, out, workspace, workspace_bytes, status, stream);
+}
+
+extern "C" int gqa_kv_append_fp8(const void *k_new, const void *v_new, gqa_dtype_t new_dtype,
+                                 void *k_cache, void *v_cache, const float *k_scale,
+                                 const float *v_scale, int32_t *seq_lens, int B, int H_kv, int d,
+                                 int L_max, int32_t *status, cudaStream_t stream) {
+    if (!k_new || !v_new || !k_cache || !v_cache || !k_scale || !v_scale || !seq_lens)
+        return GQA_ERR_NULL;
+    if (new_dtype != GQA_DTYPE_F32 && new_dtype != GQA_DTYPE_BF16) return GQA_ERR_UNSUPPORTED_DTYPE;
+    if (B <= 0 || H_kv <= 0 || L_max <= 0 || static_cast<long long>(B) * H_kv > (1ll << 30))
+        return GQA_ERR_SHAPE;
+    if (d != 64 && d != 128) return GQA_ERR_UNSUPPORTED_DIM;
+    if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(k_cache, 16) ||
+        !aligned(v_cache, 16) || !aligned(k_scale, 4) || !aligned(v_scale, 4) ||
+        !aligned(seq_lens, 4) || (status && !aligned(status, 4)))
+        return GQA_ERR_ALIGNMENT;
+    int dev = 0;
+    if (current_sm_count(&dev) <= 0) return GQA_ERR_NO_DEVICE;
+    return launch_append_fp8(k_new, v_new, new_dtype == GQA_DTYPE_BF16, k_cache, v_cache, k_scale,
+                             v_scale, seq_lens, nullptr, 0, 0, 0, B, H_kv, d, L_max, 1, status,
+                             stream);
+}
+
+extern "C" int gqa_kv_append_paged_fp8(const void *k_new, const void *v_new, gqa_dtype_t new_dtype,
+                                       void *k_pool, void *v_pool, const float *k_scale,
+                                       const float *v_scale, const int32_t *block_table,
+                                       int max_pages, int32_t *seq_lens, int B, int H_kv, int d,
+                                       int page_size, int n_pages, int32_t *status,
+                                       cudaStream_t stream) {
+    if (!k_new || !v_new || !k_pool || !v_pool || !k_scale || !v_scale || !block_table || !seq_lens)
+        return GQA_ERR_NULL;
+    if (new_dtype != GQA_DTYPE_F32 && new_dtype != GQA_DTYPE_BF16) return GQA_ERR_UNSUPPORTED_DTYPE;
+    if (B <= 0 || H_kv <= 0 || max_pages <= 0 || n_pages <= 0 || page_size <= 0 ||
+        page_size % 8 != 0 || static_cast<long long>(max_pages) * page_size > (1ll << 30) ||
+        static_cast<long long>(B) * H_kv > (1ll << 30))
+        return GQA_ERR_SHAPE;
+    if (d != 64 && d != 128) return GQA_ERR_UNSUPPORTED_DIM;
+    if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(k_pool, 16) ||
+        !aligned(v_pool, 16) || !aligned(k_scale, 4) || !aligned(v_scale, 4) ||
+        !aligned(block_table, 4) || !aligned(seq_lens, 4) || (status && !aligned(status, 4)))
+        return GQA_ERR_ALIGNMENT;
+    int dev = 0;
+    if (current_sm_count(&dev) <= 0) return GQA_ERR_NO_DEVICE;
+    return launch_append_fp8(k_new, v_new, new_dtype == GQA_DTYPE_BF16, k_pool, v_pool, k_scale,
+                             v_scale, seq_lens, block_table, max_pages, page_size, n_pages, B,
+                             H_kv, d, 0, 1, status, stream);
+}
+
+extern "C" int gqa_decode_fp8(const void *q, const void *k_cache, const void *v_cache,
+                              const float *k_scale, const float *v_scale, const int32_t *seq_lens,
+                              int B, int H_q, int H_kv, int d, int L_max, int window, float scale,
+                              float *out, void *workspace, size_t workspace_bytes,
+                              int32_t *status, cudaStream_t stream) {
+    if (!k_scale || !v_scale) return GQA_ERR_NULL;
+    if (window < 0) return GQA_ERR_SHAPE;
+    return decode_impl(q, k_cache, v_cache, seq_lens, B, H_q, H_kv, d, L_max, window, scale,
+                       GQA_DTYPE_E4M3, out, workspace, workspace_bytes, status, stream,
+                       PagedArgs(), 1, k_scale, v_scale);
+}
+
+extern "C" int gqa_decode_paged_fp8(const void *q, const void *k_pool, const void *v_pool,
+                                    const float *k_scale, const float *v_scale,
+                                    const int32_t *block_table, int max_pages,
+                                    const int32_t *seq_lens, int B, int H_q, int H_kv, int d,
+                                    int page_size, int n_pages, float scale, float *out,
+                                    void *workspace, size_t workspace_bytes, int32_t *status,
+                                    cudaStream_t stream) {
+    if (!block_table || !k_scale || !v_scale) return GQA_ERR_NULL;
+    if (!aligned(block_table, 4)) return GQA_ERR_ALIGNMENT;
+    if (max_pages <= 0 || n_pages <= 0 || page_size <= 0 || page_size % 8 != 0 ||
+        static_cast<long long>(max_pages) * page_size > (1ll << 30))
+        return GQA_ERR_SHAPE;
+    // a tile (256 or 128 rows) must lie in one page or cover whole pages
+    if (256 % page_size != 0 && page_size % 256 != 0) return GQA_ERR_SHAPE;
+    PagedArgs pg;
+    pg.block_table = block_table;
+    pg.max_pages = max_pages;
+    pg.page_size = page_size;
+    pg.n_pages = n_pages;
+    return decode_impl(q, k_pool, v_pool, seq_lens, B, H_q, H_kv, d, max_pages * page_size, 0,
+                       scale, GQA_DTYPE_E4M3, out, workspace, workspace_bytes, status, stream,
+                       pg, 1, k_scale, v_scale);
 }
 
 extern "C" const char *gqa_status_string(int code) {

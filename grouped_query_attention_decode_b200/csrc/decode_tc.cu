@@ -125,43 +125,6 @@ __device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t bytes) {
     return desc + static_cast<uint64_t>(bytes >> 4);
 }
 
-// Tiles ahead of the copy at which the paged producer loads page ids.
-constexpr int kPageAhead = 2;
-
-// A cursor over the tiles of a CTA's range, one tile at a time, used to look up page ids ahead
-// of the tile being copied.
-struct TileCursor {
-    SegmentWalker w;
-    Segment sg;
-    int jj;
-    bool live;
-
-    __device__ void init(const DecodeParams &p, const CtaRange &cr) {
-        w.init(p, cr);
-        live = w.next(sg);
-        jj = 0;
-    }
-    __device__ void advance() {
-        if (live && ++jj >= sg.len) {
-            live = w.next(sg);
-            jj = 0;
-        }
-    }
-    // Page holding box `box` of the current tile (boxes as the producer cuts them: T / boxr
-    // boxes of min(page_size, T) rows for a full tile, 8-row boxes for a partial one); 0 past
-    // the last box or the last tile.  Every box starts below the sequence's length, so the
-    // block-table index stays below max_pages.
-    __device__ int page_of_box(const DecodeParams &p, int T, int box) const {
-        if (!live) return 0;
-        const int row0 = sg.first + (sg.j0 + jj) * T;
-        const int rows = min(T, sg.n - row0);
-        const int boxr = rows == T ? min(p.page_size, T) : 8;
-        const int nbox = rows == T ? T / boxr : (rows + 7) >> 3;
-        if (box >= nbox) return 0;
-        return __ldg(p.block_table + static_cast<long long>(sg.b) * p.max_pages + (row0 + box * boxr) / p.page_size);
-    }
-};
-
 template <int D, int NH, bool PAGED>
 __global__ void __launch_bounds__(TcCfg<D, NH>::THREADS, 1)
 split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,

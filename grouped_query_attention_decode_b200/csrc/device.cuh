@@ -235,6 +235,75 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_ma
            (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, 8-bit float inputs (kind::f8f6f4), fp32 D.
+__device__ __forceinline__ void umma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                        uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// UMMA instruction descriptor for kind::f8f6f4 with e4m3 A and B (format 0), fp32 D; the
+// other fields as in idesc_bf16_f32.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N, bool a_mn_major,
+                                                      bool b_mn_major) {
+    return (1u << 4) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
+           (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// ------------------------------------------------------------------ e4m3 conversions (PTX cvt)
+// Two floats to one e4m3x2 (e0 in the low byte), round to nearest even, saturating to +-448.
+__device__ __forceinline__ uint16_t e4m3x2_from_f32(float e0, float e1) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(e1), "f"(e0));
+    return r;
+}
+
+// f16x2 (element 0 in the low half) to e4m3x2, round to nearest even, saturating.
+__device__ __forceinline__ uint16_t e4m3x2_from_f16x2(uint32_t h) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(r) : "r"(h));
+    return r;
+}
+
+// e4m3x2 to f16x2 (exact: every e4m3 value is an f16 value).
+__device__ __forceinline__ uint32_t f16x2_from_e4m3x2(uint16_t e) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(e));
+    return r;
+}
+
+// Two floats to f16x2 (e0 in the low half), round to nearest even.
+__device__ __forceinline__ uint32_t f16x2_from_f32(float e0, float e1) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(e1), "f"(e0));
+    return r;
+}
+
+// a - b and a * b on f16x2, round to nearest even (subnormals kept).
+__device__ __forceinline__ uint32_t f16x2_sub(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+__device__ __forceinline__ uint32_t f16x2_mul(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+// The two halves of an f16x2 as floats (exact).
+__device__ __forceinline__ float2 f32x2_from_f16x2(uint32_t h) {
+    float lo, hi;
+    asm("{\n\t.reg .f16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}"
+        : "=f"(lo), "=f"(hi)
+        : "r"(h));
+    return make_float2(lo, hi);
+}
+
 // ---------------------------------------------------------------------------------- misc
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;

@@ -21,6 +21,15 @@ int tc_q_box_rows(int heads_per_unit);
 int launch_split_f32(const DecodeParams &p, const float *q, const float *kc, const float *vc,
                      cudaStream_t stream);
 int launch_combine(const DecodeParams &p, cudaStream_t stream);
+// FP8 (e4m3) cache: the split kernel (K/V maps of uint8 codes with box rows tc8_tile_rows or
+// the page size, and 8-row boxes; q is read from global memory) and the quantising append.
+int tc8_tile_rows(int heads_per_unit);
+int launch_split_tc8(const TmaMaps &maps, const void *q, const DecodeParams &p, cudaStream_t stream);
+int launch_append_fp8(const void *k_new, const void *v_new, bool bf16_in, void *k_cache,
+                      void *v_cache, const float *k_scale, const float *v_scale, int32_t *seq_lens,
+                      const int32_t *block_table, int max_pages, int page_size, int n_pages,
+                      int B, int H_kv, int d, int L_max, int rows, int32_t *status,
+                      cudaStream_t stream);
 int launch_append_paged(const void *k_new, const void *v_new, void *k_pool, void *v_pool,
                         const int32_t *block_table, int max_pages, int32_t *seq_lens, int B,
                         int H_kv, int row_bytes, int page_size, int n_pages, int32_t *status,

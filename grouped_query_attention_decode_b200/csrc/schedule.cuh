@@ -41,6 +41,9 @@ struct DecodeParams {
     // max_pages * page_size.
     const int32_t *block_table;
     int max_pages, page_size, n_pages;
+    // FP8 (e4m3) cache: a code of key/value head g stands for value(code) * k_scale[g] (K)
+    // or value(code) * v_scale[g] (V); nullptr for 16- and 32-bit caches.
+    const float *k_scale, *v_scale;
     float scale_log2;                 // softmax scale * log2(e)
     unsigned long long wait_ns;       // bound of every pipeline wait
     long long slot_floats;            // RB * (d + 2)
@@ -212,6 +215,43 @@ struct SegmentWalker {
         s.whole = (j0 == 0 && len == nt);
         t += len;
         return true;
+    }
+};
+
+// Tiles ahead of the copy at which the paged producer loads page ids.
+constexpr int kPageAhead = 2;
+
+// A cursor over the tiles of a CTA's range, one tile at a time, used to look up page ids ahead
+// of the tile being copied.
+struct TileCursor {
+    SegmentWalker w;
+    Segment sg;
+    int jj;
+    bool live;
+
+    __device__ void init(const DecodeParams &p, const CtaRange &cr) {
+        w.init(p, cr);
+        live = w.next(sg);
+        jj = 0;
+    }
+    __device__ void advance() {
+        if (live && ++jj >= sg.len) {
+            live = w.next(sg);
+            jj = 0;
+        }
+    }
+    // Page holding box `box` of the current tile (boxes as the producer cuts them: T / boxr
+    // boxes of min(page_size, T) rows for a full tile, 8-row boxes for a partial one); 0 past
+    // the last box or the last tile.  Every box starts below the sequence's length, so the
+    // block-table index stays below max_pages.
+    __device__ int page_of_box(const DecodeParams &p, int T, int box) const {
+        if (!live) return 0;
+        const int row0 = sg.first + (sg.j0 + jj) * T;
+        const int rows = min(T, sg.n - row0);
+        const int boxr = rows == T ? min(p.page_size, T) : 8;
+        const int nbox = rows == T ? T / boxr : (rows + 7) >> 3;
+        if (box >= nbox) return 0;
+        return __ldg(p.block_table + static_cast<long long>(sg.b) * p.max_pages + (row0 + box * boxr) / p.page_size);
     }
 };
 

@@ -11,6 +11,10 @@ Recipe (all draws from one ``torch.Generator('cpu')`` seeded with the workload's
   5. v_new    [B, H_kv, d]           same
   6. lengths  [B]  either the fixed length, or uniform integers in [1, L_max] (ragged)
 Each float is drawn in fp32 and rounded to the storage dtype with round-to-nearest-even.
+An FP8 (e4m3) cache (``kv_format="e4m3"``) first draws k_scale, v_scale [H_kv] =
+kv_std * U(0.75, 1.25) / 32; its cache steps 2-3 draw N(0, 1) * 32 and round it to the nearest
+e4m3 code (torch's float8_e4m3fn), so code * scale is again ~ N(0, kv_std^2); q, k_new and v_new
+stay in the workload's dtype (bf16) and the append quantises the new rows.
 ``lengths`` is the number of rows attended AFTER this step's append, so the cache starts with
 ``seq_lens = lengths - 1`` and the append writes row ``lengths - 1``.  With Q > 1 query tokens
 per sequence (speculative verification), q is [B, Q, H_q, d], k_new/v_new are [B, Q, H_kv, d]
@@ -43,6 +47,7 @@ class Workload:
     window: int = 0                    # > 0: sliding window, attend the last `window` rows
     page_size: int = 0                 # > 0: the cache lives in a paged pool (see make_paged)
     queries: int = 1                   # query tokens per sequence (speculative verification)
+    kv_format: str = ""                # "e4m3": FP8 cache codes with per-head scales
     note: str = field(default="", compare=False)
 
     @property
@@ -51,7 +56,14 @@ class Workload:
 
     @property
     def elem_bytes(self) -> int:
+        """Bytes of one cached K or V element."""
+        if self.kv_format == "e4m3":
+            return 1
         return torch.tensor([], dtype=self.dtype).element_size()
+
+    @property
+    def fp8(self) -> bool:
+        return self.kv_format == "e4m3"
 
 
 # The pages' workloads, each named by what it is.
@@ -87,16 +99,31 @@ WORKLOADS = {
         Workload("ragged_long_window4096", B=32, H_q=32, H_kv=8, d=128, L_max=32768,
                  dtype=torch.bfloat16, q_std=1.0, kv_std=1.0, seed=4, length=None, window=4096,
                  note="the ragged batch with a Mistral-style sliding window of 4096 rows"),
+        Workload("llama2_70b_layer_fp8", B=16, H_q=64, H_kv=8, d=128, L_max=4096,
+                 dtype=torch.bfloat16, q_std=0.5, kv_std=0.5, seed=1, length=4096, kv_format="e4m3",
+                 note="the Llama-2-70B-shaped layer with an FP8 (e4m3) cache"),
+        Workload("ragged_long_fp8", B=32, H_q=32, H_kv=8, d=128, L_max=32768, dtype=torch.bfloat16,
+                 q_std=1.0, kv_std=1.0, seed=4, length=None, kv_format="e4m3",
+                 note="the ragged long-context batch with an FP8 (e4m3) cache"),
     ]
 }
 
 
 def custom(name="custom", *, B, H_q, H_kv, d, L_max, dtype=torch.bfloat16, q_std=1.0,
            kv_std=1.0, seed=1234, length=None, scale=None, window=0, page_size=0,
-           queries=1) -> Workload:
+           queries=1, kv_format="") -> Workload:
     return Workload(name, B=B, H_q=H_q, H_kv=H_kv, d=d, L_max=L_max, dtype=dtype, q_std=q_std,
                     kv_std=kv_std, seed=seed, length=length, scale=scale, window=window,
-                    page_size=page_size, queries=queries)
+                    page_size=page_size, queries=queries, kv_format=kv_format)
+
+
+E4M3_NAN = 0x7F
+
+
+def _e4m3_codes(shape, gen) -> torch.Tensor:
+    """uint8 e4m3 codes of N(0, 1) * 32 rounded to nearest (torch's float8_e4m3fn)."""
+    x = torch.randn(shape, generator=gen, dtype=torch.float32).mul_(32.0).clamp_(-448.0, 448.0)
+    return x.to(torch.float8_e4m3fn).view(torch.uint8)
 
 
 def _normal(shape, gen, std, dtype):
@@ -117,12 +144,24 @@ def make_inputs(w: Workload, lengths=None, poison: bool = False) -> dict:
     g.manual_seed(w.seed)
     Qn = w.queries
     q = _normal((w.B, w.H_q, w.d) if Qn == 1 else (w.B, Qn, w.H_q, w.d), g, w.q_std, w.dtype)
-    k_cache = torch.empty((w.B, w.L_max, w.H_kv, w.d), dtype=w.dtype)
-    v_cache = torch.empty_like(k_cache)
-    for b in range(w.B):
-        k_cache[b] = _normal((w.L_max, w.H_kv, w.d), g, w.kv_std, w.dtype)
-    for b in range(w.B):
-        v_cache[b] = _normal((w.L_max, w.H_kv, w.d), g, w.kv_std, w.dtype)
+    extra = {}
+    if w.fp8:
+        u = torch.rand((2, w.H_kv), generator=g, dtype=torch.float32)
+        extra["k_scale"] = (w.kv_std * (0.75 + 0.5 * u[0]) / 32.0).float()
+        extra["v_scale"] = (w.kv_std * (0.75 + 0.5 * u[1]) / 32.0).float()
+        k_cache = torch.empty((w.B, w.L_max, w.H_kv, w.d), dtype=torch.uint8)
+        v_cache = torch.empty_like(k_cache)
+        for b in range(w.B):
+            k_cache[b] = _e4m3_codes((w.L_max, w.H_kv, w.d), g)
+        for b in range(w.B):
+            v_cache[b] = _e4m3_codes((w.L_max, w.H_kv, w.d), g)
+    else:
+        k_cache = torch.empty((w.B, w.L_max, w.H_kv, w.d), dtype=w.dtype)
+        v_cache = torch.empty_like(k_cache)
+        for b in range(w.B):
+            k_cache[b] = _normal((w.L_max, w.H_kv, w.d), g, w.kv_std, w.dtype)
+        for b in range(w.B):
+            v_cache[b] = _normal((w.L_max, w.H_kv, w.d), g, w.kv_std, w.dtype)
     new_shape = (w.B, w.H_kv, w.d) if Qn == 1 else (w.B, Qn, w.H_kv, w.d)
     k_new = _normal(new_shape, g, w.kv_std, w.dtype)
     v_new = _normal(new_shape, g, w.kv_std, w.dtype)
@@ -135,13 +174,13 @@ def make_inputs(w: Workload, lengths=None, poison: bool = False) -> dict:
         assert drawn.shape == (w.B,)
     seq_lens_pre = torch.clamp(drawn - Qn, min=0).to(torch.int32)
     if poison:
-        nan = float("nan")
+        nan = E4M3_NAN if w.fp8 else float("nan")
         for b in range(w.B):
             k_cache[b, int(seq_lens_pre[b]):] = nan
             v_cache[b, int(seq_lens_pre[b]):] = nan
     return {
         "q": q, "k_cache": k_cache, "v_cache": v_cache, "k_new": k_new, "v_new": v_new,
-        "seq_lens_pre": seq_lens_pre, "lengths": drawn, "scale": w.softmax_scale,
+        "seq_lens_pre": seq_lens_pre, "lengths": drawn, "scale": w.softmax_scale, **extra,
     }
 
 
@@ -158,8 +197,9 @@ def make_paged(x: dict, page_size: int, extra_pages: int = 3, seed: int = 99) ->
     g = torch.Generator(device="cpu")
     g.manual_seed(seed)
     perm = torch.randperm(n_pages, generator=g)[: B * max_pages].to(torch.int32)
-    k_pool = torch.full((n_pages, page_size, H_kv, d), float("nan"), dtype=kc.dtype)
-    v_pool = torch.full_like(k_pool, float("nan"))
+    nan = E4M3_NAN if kc.dtype == torch.uint8 else float("nan")  # unused pages hold NaN
+    k_pool = torch.full((n_pages, page_size, H_kv, d), nan, dtype=kc.dtype)
+    v_pool = torch.full_like(k_pool, nan)
     k_pool[perm.long()] = kc.reshape(B * max_pages, page_size, H_kv, d)
     v_pool[perm.long()] = vc.reshape(B * max_pages, page_size, H_kv, d)
     return {"k_pool": k_pool, "v_pool": v_pool, "block_table": perm.reshape(B, max_pages).contiguous()}

@@ -52,7 +52,9 @@ extern "C" {
 /* Element type of q, k_new, v_new, k_cache and v_cache. */
 typedef enum {
     GQA_DTYPE_F32 = 0,  /* IEEE float32; computed on CUDA cores in float32 */
-    GQA_DTYPE_BF16 = 1  /* bfloat16; products on tcgen05 tensor cores, float32 accumulation */
+    GQA_DTYPE_BF16 = 1, /* bfloat16; products on tcgen05 tensor cores, float32 accumulation */
+    GQA_DTYPE_E4M3 = 2  /* FP8 cache (the *_fp8 calls only): e4m3 codes with per-head scales,
+                           bfloat16 q; accepted by gqa_decode_workspace_size */
 } gqa_dtype_t;
 
 /* Return codes. */
@@ -201,6 +203,54 @@ int gqa_decode_paged(const void *q, const void *k_pool, const void *v_pool,
                      int H_q, int H_kv, int d, int page_size, int n_pages, float scale,
                      gqa_dtype_t dtype, float *out, void *workspace, size_t workspace_bytes,
                      int32_t *status, cudaStream_t stream);
+
+/*
+ * FP8 (e4m3) KV cache with one scale per key/value head.  "GQA 阅读笔记", section
+ * "复现性与工程实践", mixed-precision item: serving systems store the KV cache in FP8, which
+ * halves the per-step KV bytes of a 16-bit cache (GQA-8 with FP8 reads 16x fewer bytes than
+ * MHA with FP16); the FlashAttention-2 GQA article (intelliparadigm.com), section 4.2 item 3,
+ * stores the cache in FP8 and dequantises it when read.  The pages fix neither the format nor
+ * the scaling; this library reads them as:
+ *   - the cache holds OCP FP8 E4M3 codes (1 sign, 4 exponent bits with bias 7, 3 mantissa
+ *     bits, no infinities, 0x7F / 0xFF NaN, largest finite magnitude 448), one byte per element,
+ *     in the layouts of the 16-bit calls: k_cache, v_cache [B][L_max][H_kv][d] uint8, or the
+ *     paged pools [n_pages][page_size][H_kv][d] uint8;
+ *   - k_scale, v_scale [H_kv] float32 (device): code c of key/value head g stands for
+ *     value(c) * k_scale[g] in K and value(c) * v_scale[g] in V;
+ *   - q is bfloat16 [B][H_q][d]; out is float32.
+ *
+ * gqa_kv_append_fp8 / gqa_kv_append_paged_fp8: the append of gqa_kv_append / gqa_kv_append_paged
+ *   with quantisation: element x of head g of k_new (v_new) is stored as the e4m3 code nearest
+ *   to the float32 quotient x / k_scale[g] (x / v_scale[g]); ties go to the even mantissa and
+ *   magnitudes past 448 saturate to +-448.  k_new, v_new [B][H_kv][d] are `new_dtype`
+ *   (GQA_DTYPE_BF16 or GQA_DTYPE_F32).  Overflow and page errors as the 16-bit calls.
+ * gqa_decode_fp8: gqa_decode (window = 0) or gqa_decode_window (window >= 1) over the e4m3
+ *   cache: the attention of the dequantised values.  Workspace: gqa_decode_workspace_size(...,
+ *   GQA_DTYPE_E4M3).  Accuracy: the scores and the softmax weights enter the tensor cores as
+ *   several e4m3 terms (q to its full bfloat16 precision, the weights to ~12 significant
+ *   bits), with float32 accumulation.
+ * gqa_decode_paged_fp8: the paged decode over e4m3 pools; page_size a multiple of 8 that
+ *   divides 256 or is a multiple of 256.
+ * Scales must be positive and finite (not checked).  NULL scales give GQA_ERR_NULL.
+ */
+int gqa_kv_append_fp8(const void *k_new, const void *v_new, gqa_dtype_t new_dtype, void *k_cache,
+                      void *v_cache, const float *k_scale, const float *v_scale,
+                      int32_t *seq_lens, int B, int H_kv, int d, int L_max, int32_t *status,
+                      cudaStream_t stream);
+int gqa_kv_append_paged_fp8(const void *k_new, const void *v_new, gqa_dtype_t new_dtype,
+                            void *k_pool, void *v_pool, const float *k_scale,
+                            const float *v_scale, const int32_t *block_table, int max_pages,
+                            int32_t *seq_lens, int B, int H_kv, int d, int page_size,
+                            int n_pages, int32_t *status, cudaStream_t stream);
+int gqa_decode_fp8(const void *q, const void *k_cache, const void *v_cache, const float *k_scale,
+                   const float *v_scale, const int32_t *seq_lens, int B, int H_q, int H_kv, int d,
+                   int L_max, int window, float scale, float *out, void *workspace,
+                   size_t workspace_bytes, int32_t *status, cudaStream_t stream);
+int gqa_decode_paged_fp8(const void *q, const void *k_pool, const void *v_pool,
+                         const float *k_scale, const float *v_scale, const int32_t *block_table,
+                         int max_pages, const int32_t *seq_lens, int B, int H_q, int H_kv, int d,
+                         int page_size, int n_pages, float scale, float *out, void *workspace,
+                         size_t workspace_bytes, int32_t *status, cudaStream_t stream);
 
 /*
  * gqa_decode_noalloc: gqa_decode without a caller-provided workspace.  (The pages have no
