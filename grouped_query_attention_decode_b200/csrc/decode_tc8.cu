@@ -68,7 +68,9 @@ struct Tc8Cfg {
     static constexpr uint32_t IDESC_PV = idesc_e4m3_f32(D, 3 * RP, true, true);
     static constexpr int NWG = NH >= 32 ? NH / 16 : 1;
     static constexpr int NHW = NH / NWG;
-    static constexpr int THREADS = 64 + 128 * NWG;
+    // NH <= 8: two warpgroups take alternate tiles (their softmax chains overlap)
+    static constexpr int PP = NH <= 8 ? 2 : 1;
+    static constexpr int THREADS = 64 + 128 * NWG * PP;
     static constexpr int NHW4 = (NHW + 3) / 4;
     static constexpr int LOG2NHW = NHW >= 16 ? 4 : NHW >= 8 ? 3 : NHW >= 4 ? 2 : NHW >= 2 ? 1 : 0;
 
@@ -82,9 +84,11 @@ struct Tc8Cfg {
         int b0;
         int pad_;
         long long begin, end, off0;
-        float qf[2][RP];                    // 1 / c_h of each column of the unit's q buffer
-        float4 wmax[NWG][2][4][NHW4];
-        float lsum[NWG][4][NHW];
+        float qf[2][RP];                    // score factor of each column: scale * k_scale / c_h
+        float vsc[2];                       // v_scale of the unit's key/value head
+        float4 wmax[NWG * PP][2][4][NHW4];
+        float lsum[NWG * PP][4][NHW];
+        float mx[NHW];                      // running maximum handed over (PP = 2)
     };
 
     static constexpr int SMEM_LIMIT = 232448;
@@ -95,6 +99,9 @@ struct Tc8Cfg {
     static constexpr int S = S_FIT > 8 ? 8 : S_FIT;
     static constexpr int SMEM_BYTES = S * STAGE_BYTES + FIXED;
     static_assert(S >= 2, "shared memory too small for a double-buffered ring");
+    static_assert(!(D == 128 && T == 256) || S >= 3, "64 KB stages: keep three in the ring");
+    static_assert(PP == 1 || NHW * D * 4 <= P_BYTES, "hand-over area must fit in a P buffer");
+    static_assert(PP == 1 || NWG == 1, "alternate-tile warpgroups only with one head slice");
     static_assert(Q8_BYTES % 1024 == 0 && P_BYTES % 1024 == 0 && STAGE_BYTES % 1024 == 0, "");
 };
 
@@ -190,7 +197,7 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         for (int j = 0; j < 2; ++j) {
             mbar_init(&sm->q_full[j], 1);
             mbar_init(&sm->q_empty[j], 1);               // the unit's last S^T has been computed
-            mbar_init(&sm->qf_empty[j], 4 * C::NWG);     // every softmax warp read the 1/c_h
+            mbar_init(&sm->qf_empty[j], 4 * C::NWG * C::PP);  // every softmax warp read the factors
             mbar_init(&sm->s_full[j], 1);
             mbar_init(&sm->s_empty[j], 4 * C::NWG);
             mbar_init(&sm->p_full[j], 4 * C::NWG);
@@ -267,14 +274,16 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         }
         // q of the current unit -> rows [q_hi | q_lo] of the unit's q buffer (K-major, swizzled
         // like the cache tiles) and 1/c_h per column.  8 lanes per q row, D/8 elements each.
-        auto convert_q = [&](int qb) {
+        auto convert_q = [&](int qb, const Segment &su) {
             constexpr int V = D / 8;
             uint8_t *q8 = q8_base + qb * C::Q8_BYTES;
             const int sub = lane >> 3, seg = lane & 7;
+            const float kfac = p.scale_log2 * p.k_scale[su.kvh];
+            if (lane == 0) sm->vsc[qb] = p.v_scale[su.kvh];
 #pragma unroll 1
             for (int r0 = 0; r0 < RP; r0 += 4) {
                 const int rr = r0 + sub;
-                const long long qrow = rr < p.RB ? out_row(p, sg.b, sg.kvh, sg.hb, rr) : -1;
+                const long long qrow = rr < p.RB ? out_row(p, su.b, su.kvh, su.hb, rr) : -1;
                 float v[V];
                 if (qrow >= 0) {
                     const uint4 *src = reinterpret_cast<const uint4 *>(q + qrow * D + seg * V);
@@ -325,7 +334,7 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                     *reinterpret_cast<uint2 *>(q8 + kmajor_chunk<ROWB>(rr, seg >> 1) + half) = make_uint2(hw[0], hw[1]);
                     *reinterpret_cast<uint2 *>(q8 + kmajor_chunk<ROWB>(RP + rr, seg >> 1) + half) = make_uint2(lw[0], lw[1]);
                 }
-                if (seg == 0) sm->qf[qb][rr] = __uint_as_float(static_cast<uint32_t>(127 - sh) << 23);
+                if (seg == 0) sm->qf[qb][rr] = kfac * __uint_as_float(static_cast<uint32_t>(127 - sh) << 23);
             }
             fence_proxy_async_smem();
             __syncwarp();
@@ -342,9 +351,15 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 break;
             }
             ++sidx;
-            // The conversion waits on global loads: do it when the ring is full (before the
-            // first wait for a free stage), or once the unit's tiles are all issued.
+            // The conversion waits on global loads.  The CTA's first unit converts before any
+            // tile is requested (its loads would otherwise queue behind every CTA's first
+            // stages); later units convert when the ring is full (before the first wait for a
+            // free stage), or once their tiles are all issued.
             bool q_pending = true;
+            if (i == 0) {
+                convert_q(qb, sg);
+                q_pending = false;
+            }
             for (int jj = 0; jj < sg.len; ++jj) {
                 const int st = i % S;
                 const int row0 = sg.first + (sg.j0 + jj) * T;
@@ -358,7 +373,7 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                     ahead.advance();
                 }
                 if (q_pending && i >= S) {
-                    convert_q(qb);
+                    convert_q(qb, sg);
                     q_pending = false;
                 }
                 got = true;
@@ -401,7 +416,7 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 }
                 ++i;
             }
-            if (ok && q_pending) convert_q(qb);
+            if (ok && q_pending) convert_q(qb, sg);
         }
         if (lane == 0) {
             if (!ok) fail();
@@ -493,14 +508,24 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         }
     } else {
         // ------------------------------------------------------------------ softmax warps
+        // NWG warpgroups split the heads (NH >= 32), or -- PP = 2, NH <= 8 -- two warpgroups
+        // take alternate tiles of the line (tile i goes to warpgroup i & 1, which also owns S,
+        // P and O buffer i & 1).  Each then keeps its own online softmax over its tiles, and at
+        // the end of a unit the second hands its state to the first, which merges the two
+        // (log-sum-exp) and writes the result.  A failed wait never makes a warpgroup leave
+        // early: it skips the remaining work and both agree at the unit's merge barrier.
         constexpr int NHW = C::NHW;
+        constexpr int PP = C::PP;
         constexpr int SCOLS = C::NWG == 1 ? RP : NHW;
-        const int wg = (warp - 2) >> 2;
+        const int wgi = (warp - 2) >> 2;              // 0 .. NWG * PP - 1
+        const int pp = PP == 2 ? wgi : 0;             // tile parity taken (PP = 2)
+        const int wg = PP == 2 ? 0 : wgi;             // head slice
         const int hbase = wg * NHW;
-        const uint32_t bar_id = 1 + wg;
+        const uint32_t bar_id = 1 + wgi;
+        const uint32_t bar_pair = 1 + C::NWG * PP;    // both tile warpgroups (PP = 2)
         const int q4 = warp & 3;
         const int row = q4 * 32 + lane;          // row of each 128-row half of the tile
-        const int sm_tid = threadIdx.x - 64;
+        const int sm_tid = threadIdx.x - 64 - 128 * pp;
         const uint32_t lane_addr = static_cast<uint32_t>(q4 * 32) << 16;
         const int dcol = (D == 128) ? row : (lane < 16 ? q4 * 16 + lane : -1);
         SegmentWalker w;
@@ -509,6 +534,32 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         int i = 0, sidx = 0;
         bool ok = true;
         float O[NHW], l[NHW], m_run[NHW], alpha[NHW], f[NHW];
+        // O of tile t (this warpgroup's) folded into the running sum, scaled by `scale_by`
+        auto fold_o = [&](int t, const float *scale_by) -> bool {
+            const int ob = t % C::OB;
+            if (!wait_bounded(&sm->o_full[ob], (t / C::OB) & 1, abort_flag, budget)) return false;
+            tc_fence_after_sync();
+            const uint32_t obase = tmem + lane_addr + C::O_COL + ob * 3 * RP + hbase;
+#pragma unroll
+            for (int c = 0; c < NHW; c += 16) {
+                uint32_t hi[16], mi[16], lo[16];
+                tmem_ld16(obase + c, hi);
+                tmem_ld16(obase + RP + c, mi);
+                tmem_ld16(obase + 2 * RP + c, lo);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    if (c + e < NHW) {
+                        const float o = __uint_as_float(hi[e]) + 0.0625f * __uint_as_float(mi[e]) +
+                                        0.00390625f * __uint_as_float(lo[e]);
+                        O[c + e] = scale_by != nullptr ? (O[c + e] + o) * scale_by[c + e] : O[c + e] + o;
+                    }
+            }
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm->o_empty[ob]);
+            return true;
+        };
         while (ok && w.next(sg)) {
 #pragma unroll
             for (int h = 0; h < NHW; ++h) {
@@ -517,13 +568,14 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 m_run[h] = -INFINITY;
             }
             bool bad = false;
-            // The unit's score factors: softmax scale (log2) * k_scale[g] / c_h.
+            // The unit's score factors (softmax scale in log2 units * k_scale[g] / c_h) and
+            // v_scale[g], written by the producer with the converted q.
             const int qb = sidx % C::QB;
-            const float ks = p.k_scale[sg.kvh];
-            const float vs = p.v_scale[sg.kvh];
+            float vs = 0.f;
             if (wait_bounded(&sm->q_full[qb], (sidx / C::QB) & 1, abort_flag, budget)) {
 #pragma unroll
-                for (int h = 0; h < NHW; ++h) f[h] = p.scale_log2 * ks * sm->qf[qb][hbase + h];
+                for (int h = 0; h < NHW; ++h) f[h] = sm->qf[qb][hbase + h];
+                vs = sm->vsc[qb];
             } else {
                 bad = true;
 #pragma unroll
@@ -532,14 +584,17 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm->qf_empty[qb]);
             ++sidx;
+            int prev_t = -1;  // this warpgroup's previous tile in the unit
             for (int jj = 0; jj < sg.len; ++jj, ++i) {
+                if (PP == 2 && (i & 1) != pp) continue;
                 const int j2 = i & 1;
                 const int rows = min(T, sg.n - sg.first - (sg.j0 + jj) * T);
                 if (rows < T && !bad && wait_bounded(&sm->kv_full[i % S], (i / S) & 1, abort_flag, budget)) {
                     // Rows past n: zero V so that 0-weight rows add exactly 0.
                     uint8_t *vbase = st_base + (i % S) * C::STAGE_BYTES + C::TILE_BYTES;
                     constexpr int CPR = ROWB / 16;
-                    for (int c = sm_tid; c < (T - rows) * CPR; c += 128 * C::NWG)
+                    const int nthr = PP == 2 ? 128 : 128 * C::NWG;
+                    for (int c = sm_tid; c < (T - rows) * CPR; c += nthr)
                         *reinterpret_cast<uint4 *>(vbase + (rows + c / CPR) * ROWB + (c % CPR) * 16) = make_uint4(0, 0, 0, 0);
                 } else if (rows < T) {
                     bad = true;
@@ -592,16 +647,21 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                         }
                         warp_max_transpose8<NHW, C::LOG2NHW>(wm, lane);
                         if (lane < NHW)
-                            reinterpret_cast<float *>(&sm->wmax[wg][j2][q4][0])[transpose_head8<NHW, C::LOG2NHW>(lane)] = wm[0];
+                            reinterpret_cast<float *>(&sm->wmax[wgi][j2][q4][0])[transpose_head8<NHW, C::LOG2NHW>(lane)] = wm[0];
                     }
                     if (named_bar_any(bar_id, 128, bad)) {
-                        ok = false;
-                        break;
+                        bad = true;
+                        if constexpr (PP == 1) {
+                            ok = false;
+                            break;
+                        } else {
+                            continue;  // skip to the unit's merge barrier
+                        }
                     }
 #pragma unroll
                     for (int h4 = 0; h4 < C::NHW4; ++h4) {
-                        const float4 a = sm->wmax[wg][j2][0][h4], b = sm->wmax[wg][j2][1][h4];
-                        const float4 c = sm->wmax[wg][j2][2][h4], e = sm->wmax[wg][j2][3][h4];
+                        const float4 a = sm->wmax[wgi][j2][0][h4], b = sm->wmax[wgi][j2][1][h4];
+                        const float4 c = sm->wmax[wgi][j2][2][h4], e = sm->wmax[wgi][j2][3][h4];
                         const float t4[4] = {fmaxf(fmaxf(a.x, b.x), fmaxf(c.x, e.x)),
                                              fmaxf(fmaxf(a.y, b.y), fmaxf(c.y, e.y)),
                                              fmaxf(fmaxf(a.z, b.z), fmaxf(c.z, e.z)),
@@ -621,6 +681,13 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                     for (int h = 0; h < NHW; ++h) alpha[h] = 1.f;
                 }
 
+                // P buffer j2 last fed the PV of this warpgroup's previous tile.  With one
+                // warpgroup that PV is known complete (its O was folded during the tile in
+                // between); with two, wait for it here, or P could be overwritten under a running
+                // PV and p_full[j2] could run a phase ahead of the issuer.
+                if (PP == 2 && prev_t >= 0 && !bad &&
+                    !wait_bounded(&sm->o_full[prev_t % C::OB], (prev_t / C::OB) & 1, abort_flag, budget))
+                    bad = true;
                 // P of this thread's rows, as three e4m3 terms, one 16-byte chunk per term and
                 // row (the warpgroup's 16 heads; zero bytes for padding heads).
 #pragma unroll
@@ -640,12 +707,16 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                     uint32_t tw[3][4];
 #pragma unroll
                     for (int k = 0; k < 16; k += 4) {
-                        uint16_t a0, a1, a2, b0, b1, b2;
-                        split3(pv[k], pv[k + 1], a0, a1, a2);
-                        split3(pv[k + 2], pv[k + 3], b0, b1, b2);
-                        tw[0][k / 4] = static_cast<uint32_t>(a0) | (static_cast<uint32_t>(b0) << 16);
-                        tw[1][k / 4] = static_cast<uint32_t>(a1) | (static_cast<uint32_t>(b1) << 16);
-                        tw[2][k / 4] = static_cast<uint32_t>(a2) | (static_cast<uint32_t>(b2) << 16);
+                        if (k < NHW) {
+                            uint16_t a0, a1, a2, b0, b1, b2;
+                            split3(pv[k], pv[k + 1], a0, a1, a2);
+                            split3(pv[k + 2], pv[k + 3], b0, b1, b2);
+                            tw[0][k / 4] = static_cast<uint32_t>(a0) | (static_cast<uint32_t>(b0) << 16);
+                            tw[1][k / 4] = static_cast<uint32_t>(a1) | (static_cast<uint32_t>(b1) << 16);
+                            tw[2][k / 4] = static_cast<uint32_t>(a2) | (static_cast<uint32_t>(b2) << 16);
+                        } else {
+                            tw[0][k / 4] = tw[1][k / 4] = tw[2][k / 4] = 0u;
+                        }
                     }
                     const int trow = hf * 128 + row;
                     const uint32_t off = p_chunk<RP>(trow, hbase >> 4);
@@ -658,74 +729,69 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm->p_full[j2]);
 
-                if (jj > 0) {
-                    const int t = i - 1, ob = t % C::OB;
-                    if (!wait_bounded(&sm->o_full[ob], (t / C::OB) & 1, abort_flag, budget)) {
-                        bad = true;
-                        continue;
-                    }
-                    tc_fence_after_sync();
-                    const uint32_t obase = tmem + lane_addr + C::O_COL + ob * 3 * RP + hbase;
-#pragma unroll
-                    for (int c = 0; c < NHW; c += 16) {
-                        uint32_t hi[16], mi[16], lo[16];
-                        tmem_ld16(obase + c, hi);
-                        tmem_ld16(obase + RP + c, mi);
-                        tmem_ld16(obase + 2 * RP + c, lo);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int e = 0; e < 16; ++e)
-                            if (c + e < NHW)
-                                O[c + e] = (O[c + e] + (__uint_as_float(hi[e]) + 0.0625f * __uint_as_float(mi[e]) +
-                                                        0.00390625f * __uint_as_float(lo[e]))) * alpha[c + e];
-                    }
-                    tc_fence_before_sync();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&sm->o_empty[ob]);
-                }
+                // O of this warpgroup's previous tile was computed against the previous
+                // maximum; fold it in and move the sum to the current one.
+                if (prev_t >= 0 && !fold_o(prev_t, alpha)) bad = true;
+                prev_t = i;
             }
             if (!ok) break;
-            const int tl = i - 1, obl = tl % C::OB;
-            if (!bad && wait_bounded(&sm->o_full[obl], (tl / C::OB) & 1, abort_flag, budget)) {
-                tc_fence_after_sync();
-                const uint32_t obase = tmem + lane_addr + C::O_COL + obl * 3 * RP + hbase;
-#pragma unroll
-                for (int c = 0; c < NHW; c += 16) {
-                    uint32_t hi[16], mi[16], lo[16];
-                    tmem_ld16(obase + c, hi);
-                    tmem_ld16(obase + RP + c, mi);
-                    tmem_ld16(obase + 2 * RP + c, lo);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        if (c + e < NHW)
-                            O[c + e] += __uint_as_float(hi[e]) + 0.0625f * __uint_as_float(mi[e]) +
-                                        0.00390625f * __uint_as_float(lo[e]);
-                }
-                tc_fence_before_sync();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sm->o_empty[obl]);
-            } else {
-                bad = true;
-            }
+            if (prev_t >= 0 && (bad || !fold_o(prev_t, nullptr))) bad = true;
 #pragma unroll
             for (int h = 0; h < NHW; ++h) {
                 const float sum = warp_sum_f32(l[h]);
-                if (lane == 0) sm->lsum[wg][q4][h] = sum;
+                if (lane == 0) sm->lsum[wgi][q4][h] = sum;
             }
-            if (named_bar_any(bar_id, 128, bad)) {
-                ok = false;
-                break;
+            float Lh[NHW];
+            if constexpr (PP == 2) {
+                // The odd-tile warpgroup hands (O, m) to the even one through its own P buffer
+                // (free: its PVs are done); l went through lsum.
+                float *xo = reinterpret_cast<float *>(p_base + C::P_BYTES);
+                if (pp == 1) {
+                    if (dcol >= 0) {
+#pragma unroll
+                        for (int h = 0; h < NHW; ++h) xo[h * D + dcol] = O[h];
+                    }
+                    if (sm_tid < NHW) {
+                        float mv = -INFINITY;
+#pragma unroll
+                        for (int hh = 0; hh < NHW; ++hh)
+                            if (hh == sm_tid) mv = m_run[hh];
+                        sm->mx[sm_tid] = mv;
+                    }
+                }
+                if (named_bar_any(bar_pair, 256, bad)) {
+                    ok = false;
+                    break;
+                }
+                if (pp == 0) {
+#pragma unroll
+                    for (int h = 0; h < NHW; ++h) {
+                        const float m1 = sm->mx[h];
+                        const float L0 = sm->lsum[0][0][h] + sm->lsum[0][1][h] + sm->lsum[0][2][h] + sm->lsum[0][3][h];
+                        const float L1 = sm->lsum[1][0][h] + sm->lsum[1][1][h] + sm->lsum[1][2][h] + sm->lsum[1][3][h];
+                        const float M = fmaxf(m_run[h], m1);
+                        const float a0 = m_run[h] == -INFINITY ? 0.f : ex2_approx(m_run[h] - M);
+                        const float a1 = m1 == -INFINITY ? 0.f : ex2_approx(m1 - M);
+                        if (dcol >= 0) O[h] = O[h] * a0 + xo[h * D + dcol] * a1;
+                        Lh[h] = L0 * a0 + L1 * a1;
+                        m_run[h] = M;
+                    }
+                }
+            } else {
+                if (named_bar_any(bar_id, 128, bad)) {
+                    ok = false;
+                    break;
+                }
+#pragma unroll
+                for (int h = 0; h < NHW; ++h)
+                    Lh[h] = sm->lsum[wg][0][h] + sm->lsum[wg][1][h] + sm->lsum[wg][2][h] + sm->lsum[wg][3][h];
             }
-            if (dcol >= 0) {
+            if (pp == 0 && dcol >= 0) {
                 if (sg.whole) {
 #pragma unroll
                     for (int h = 0; h < NHW; ++h) {
                         const long long orow = out_row(p, sg.b, sg.kvh, sg.hb, hbase + h);
-                        if (orow >= 0) {
-                            const float L = sm->lsum[wg][0][h] + sm->lsum[wg][1][h] + sm->lsum[wg][2][h] + sm->lsum[wg][3][h];
-                            p.out[orow * D + dcol] = O[h] * vs / L;
-                        }
+                        if (orow >= 0) p.out[orow * D + dcol] = O[h] * vs / Lh[h];
                     }
                 } else {
                     float *slot = p.ws + p.hdr_floats +
@@ -734,17 +800,22 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                     for (int h = 0; h < NHW; ++h)
                         if (hbase + h < p.RB) slot[(hbase + h) * D + dcol] = O[h] * vs;
                     if (dcol < NHW && hbase + dcol < p.RB) {
-                        const int h = dcol;
-                        float m_final = -INFINITY;
+                        float m_final = -INFINITY, l_final = 0.f;
 #pragma unroll
                         for (int hh = 0; hh < NHW; ++hh)
-                            if (hh == h) m_final = m_run[hh];
-                        slot[p.RB * D + hbase + h] = m_final;
-                        slot[p.RB * D + p.RB + hbase + h] = sm->lsum[wg][0][h] + sm->lsum[wg][1][h] + sm->lsum[wg][2][h] + sm->lsum[wg][3][h];
+                            if (hh == dcol) {
+                                m_final = m_run[hh];
+                                l_final = Lh[hh];
+                            }
+                        slot[p.RB * D + hbase + dcol] = m_final;
+                        slot[p.RB * D + p.RB + hbase + dcol] = l_final;
                     }
                 }
             }
-            named_bar_sync(bar_id, 128);
+            // the next unit rewrites lsum (and the hand-over area) only after every thread
+            // has read it
+            if constexpr (PP == 2) named_bar_sync(bar_pair, 256);
+            else named_bar_sync(bar_id, 128);
         }
         if (!ok) fail();
     }

@@ -168,3 +168,14 @@ def test_fp8_rejects_bad_arguments():
     # the 16-bit entry points do not take the e4m3 type
     assert lib.gqa_decode(gqa._ptr(q), gqa._ptr(kc), gqa._ptr(kc), gqa._ptr(lens), 1, 8, 2, 128, 64, 0.1,
                           gqa.DTYPE_E4M3, gqa._ptr(out), gqa._ptr(ws), ws.numel(), None, gqa._stream(None)) == -5
+
+
+@pytest.mark.parametrize("shape", [(4, 32, 4), (4, 16, 4), (3, 64, 4), (2, 64, 2)],
+                         ids=lambda s: "B%d_Hq%d_Hkv%d" % s)
+def test_fp8_many_tiles_per_cta(oracle, shape):
+    # far more tiles than SMs: every CTA streams several tiles (the tile-alternating warpgroups
+    # of the small-group kernels both work), cuts units into pieces and ends on partial tiles
+    B, H_q, H_kv = shape
+    w = inputs.custom("fp8m", B=B, H_q=H_q, H_kv=H_kv, d=128, L_max=12000, kv_format="e4m3",
+                      q_std=2.0, seed=66)
+    _step(oracle, w, [12000, 11111, 9000, 10001][:B])
