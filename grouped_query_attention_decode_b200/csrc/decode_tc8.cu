@@ -68,9 +68,11 @@ struct Tc8Cfg {
     static constexpr uint32_t IDESC_PV = idesc_e4m3_f32(D, 3 * RP, true, true);
     static constexpr int NWG = NH >= 32 ? NH / 16 : 1;
     static constexpr int NHW = NH / NWG;
-    // NH <= 8: two warpgroups take alternate tiles (their softmax chains overlap)
-    static constexpr int PP = NH <= 8 ? 2 : 1;
-    static constexpr int THREADS = 64 + 128 * NWG * PP;
+    // 256-row tiles: one warpgroup per 128-row half, so every softmax thread owns one row and
+    // a tile's softmax takes the time of 128 rows
+    static constexpr int RS = RT;
+    static constexpr int NSW = NWG * RS;               // softmax warpgroups
+    static constexpr int THREADS = 64 + 128 * NSW;
     static constexpr int NHW4 = (NHW + 3) / 4;
     static constexpr int LOG2NHW = NHW >= 16 ? 4 : NHW >= 8 ? 3 : NHW >= 4 ? 2 : NHW >= 2 ? 1 : 0;
 
@@ -86,9 +88,8 @@ struct Tc8Cfg {
         long long begin, end, off0;
         float qf[2][RP];                    // score factor of each column: scale * k_scale / c_h
         float vsc[2];                       // v_scale of the unit's key/value head
-        float4 wmax[NWG * PP][2][4][NHW4];
-        float lsum[NWG * PP][4][NHW];
-        float mx[NHW];                      // running maximum handed over (PP = 2)
+        float4 wmax[NWG][2][4 * RS][NHW4];  // per head slice, S buffer, warp: warp maxima
+        float lsum[NWG][4 * RS][NHW];
     };
 
     static constexpr int SMEM_LIMIT = 232448;
@@ -100,8 +101,7 @@ struct Tc8Cfg {
     static constexpr int SMEM_BYTES = S * STAGE_BYTES + FIXED;
     static_assert(S >= 2, "shared memory too small for a double-buffered ring");
     static_assert(!(D == 128 && T == 256) || S >= 3, "64 KB stages: keep three in the ring");
-    static_assert(PP == 1 || NHW * D * 4 <= P_BYTES, "hand-over area must fit in a P buffer");
-    static_assert(PP == 1 || NWG == 1, "alternate-tile warpgroups only with one head slice");
+    static_assert(RS == 1 || NWG == 1, "row halves split only with one head slice");
     static_assert(Q8_BYTES % 1024 == 0 && P_BYTES % 1024 == 0 && STAGE_BYTES % 1024 == 0, "");
 };
 
@@ -197,12 +197,12 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         for (int j = 0; j < 2; ++j) {
             mbar_init(&sm->q_full[j], 1);
             mbar_init(&sm->q_empty[j], 1);               // the unit's last S^T has been computed
-            mbar_init(&sm->qf_empty[j], 4 * C::NWG * C::PP);  // every softmax warp read the factors
+            mbar_init(&sm->qf_empty[j], 4 * C::NSW);    // every softmax warp read the factors
             mbar_init(&sm->s_full[j], 1);
-            mbar_init(&sm->s_empty[j], 4 * C::NWG);
-            mbar_init(&sm->p_full[j], 4 * C::NWG);
+            mbar_init(&sm->s_empty[j], 4 * C::NSW);
+            mbar_init(&sm->p_full[j], 4 * C::NSW);
             mbar_init(&sm->o_full[j], 1);
-            mbar_init(&sm->o_empty[j], 4 * C::NWG);
+            mbar_init(&sm->o_empty[j], 4 * C::NWG);     // the first row half folds O
         }
         mbar_init(&sm->mma_done, 1);
         sm->abort = 0;
@@ -508,24 +508,26 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         }
     } else {
         // ------------------------------------------------------------------ softmax warps
-        // NWG warpgroups split the heads (NH >= 32), or -- PP = 2, NH <= 8 -- two warpgroups
-        // take alternate tiles of the line (tile i goes to warpgroup i & 1, which also owns S,
-        // P and O buffer i & 1).  Each then keeps its own online softmax over its tiles, and at
-        // the end of a unit the second hands its state to the first, which merges the two
-        // (log-sum-exp) and writes the result.  A failed wait never makes a warpgroup leave
-        // early: it skips the remaining work and both agree at the unit's merge barrier.
+        // Every softmax thread owns one row of each tile.  NWG warpgroups split the heads
+        // (NH >= 32, 128-row tiles), or -- 256-row tiles -- RS = 2 warpgroups split the rows:
+        // warpgroup w takes rows [128w, 128w + 128) of every tile.  The two halves share the
+        // running maximum (the warp maxima of both are exchanged) and the row sums; the first
+        // half folds the Oᵀ tiles into registers and writes the result.
         constexpr int NHW = C::NHW;
-        constexpr int PP = C::PP;
+        constexpr int RS = C::RS;
         constexpr int SCOLS = C::NWG == 1 ? RP : NHW;
-        const int wgi = (warp - 2) >> 2;              // 0 .. NWG * PP - 1
-        const int pp = PP == 2 ? wgi : 0;             // tile parity taken (PP = 2)
-        const int wg = PP == 2 ? 0 : wgi;             // head slice
+        constexpr int NBAR = 128 * RS;                // threads at the group's named barrier
+        const int wgi = (warp - 2) >> 2;              // 0 .. NSW - 1
+        const int hf = RS == 2 ? wgi : 0;             // row half
+        const int wg = RS == 2 ? 0 : wgi;             // head slice
+        const bool folds = hf == 0;                   // folds O and writes the result
         const int hbase = wg * NHW;
-        const uint32_t bar_id = 1 + wgi;
-        const uint32_t bar_pair = 1 + C::NWG * PP;    // both tile warpgroups (PP = 2)
+        const uint32_t bar_id = 1 + wg;
         const int q4 = warp & 3;
-        const int row = q4 * 32 + lane;          // row of each 128-row half of the tile
-        const int sm_tid = threadIdx.x - 64 - 128 * pp;
+        const int wq = hf * 4 + q4;                   // warp index within the group (0 .. 4RS-1)
+        const int row = q4 * 32 + lane;               // row of the tile half (TMEM lane)
+        const int trow = hf * 128 + row;              // row of the tile
+        const int sm_tid = threadIdx.x - 64 - 128 * (RS == 2 ? 0 : wg);  // 0 .. NBAR-1 in the group
         const uint32_t lane_addr = static_cast<uint32_t>(q4 * 32) << 16;
         const int dcol = (D == 128) ? row : (lane < 16 ? q4 * 16 + lane : -1);
         SegmentWalker w;
@@ -534,7 +536,7 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         int i = 0, sidx = 0;
         bool ok = true;
         float O[NHW], l[NHW], m_run[NHW], alpha[NHW], f[NHW];
-        // O of tile t (this warpgroup's) folded into the running sum, scaled by `scale_by`
+        // O of tile t folded into the running sum, scaled by `scale_by` (first row half only)
         auto fold_o = [&](int t, const float *scale_by) -> bool {
             const int ob = t % C::OB;
             if (!wait_bounded(&sm->o_full[ob], (t / C::OB) & 1, abort_flag, budget)) return false;
@@ -584,30 +586,24 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm->qf_empty[qb]);
             ++sidx;
-            int prev_t = -1;  // this warpgroup's previous tile in the unit
             for (int jj = 0; jj < sg.len; ++jj, ++i) {
-                if (PP == 2 && (i & 1) != pp) continue;
                 const int j2 = i & 1;
                 const int rows = min(T, sg.n - sg.first - (sg.j0 + jj) * T);
                 if (rows < T && !bad && wait_bounded(&sm->kv_full[i % S], (i / S) & 1, abort_flag, budget)) {
                     // Rows past n: zero V so that 0-weight rows add exactly 0.
                     uint8_t *vbase = st_base + (i % S) * C::STAGE_BYTES + C::TILE_BYTES;
                     constexpr int CPR = ROWB / 16;
-                    const int nthr = PP == 2 ? 128 : 128 * C::NWG;
-                    for (int c = sm_tid; c < (T - rows) * CPR; c += nthr)
+                    for (int c = sm_tid; c < (T - rows) * CPR; c += NBAR)
                         *reinterpret_cast<uint4 *>(vbase + (rows + c / CPR) * ROWB + (c % CPR) * 16) = make_uint4(0, 0, 0, 0);
                 } else if (rows < T) {
                     bad = true;
                 }
-                uint32_t shi[RT][SCOLS], slo[RT][SCOLS];
+                uint32_t shi[SCOLS], slo[SCOLS];
                 if (!bad && wait_bounded(&sm->s_full[j2], (i >> 1) & 1, abort_flag, budget)) {
                     tc_fence_after_sync();
-#pragma unroll
-                    for (int hf = 0; hf < RT; ++hf) {
-                        const uint32_t sc = tmem + lane_addr + (j2 * RT + hf) * 2 * RP + hbase;
-                        tmem_ld_cols<SCOLS>(sc, shi[hf]);
-                        tmem_ld_cols<SCOLS>(sc + RP, slo[hf]);
-                    }
+                    const uint32_t sc = tmem + lane_addr + (j2 * RT + hf) * 2 * RP + hbase;
+                    tmem_ld_cols<SCOLS>(sc, shi);
+                    tmem_ld_cols<SCOLS>(sc + RP, slo);
                     tmem_wait_ld();
                     tc_fence_before_sync();
                     __syncwarp();
@@ -615,57 +611,48 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 } else {
                     bad = true;
 #pragma unroll
-                    for (int hf = 0; hf < RT; ++hf)
-#pragma unroll
-                        for (int h = 0; h < SCOLS; ++h) shi[hf][h] = slo[hf][h] = 0u;
+                    for (int h = 0; h < SCOLS; ++h) shi[h] = slo[h] = 0u;
                 }
 
-                float x[RT][NHW];
+                float x[NHW];
                 bool need = false;
-#pragma unroll
-                for (int hf = 0; hf < RT; ++hf) {
-                    const int trow = hf * 128 + row;
+                {
                     const bool valid = trow < rows;
                     const int over = sg.first + (sg.j0 + jj) * T + trow - (sg.n - p.Q + 1);
                     const int min_col = over >= 0 ? (over + 1) * p.rb : 0;
 #pragma unroll
                     for (int h = 0; h < NHW; ++h) {
-                        x[hf][h] = (valid && hbase + h >= min_col)
-                                       ? (__uint_as_float(shi[hf][h]) + 0.0625f * __uint_as_float(slo[hf][h])) * f[h]
-                                       : -INFINITY;
-                        need |= x[hf][h] > m_run[h] + kLazyLog2_8;
+                        x[h] = (valid && hbase + h >= min_col)
+                                   ? (__uint_as_float(shi[h]) + 0.0625f * __uint_as_float(slo[h])) * f[h]
+                                   : -INFINITY;
+                        need |= x[h] > m_run[h] + kLazyLog2_8;
                     }
                 }
-                if (named_bar_any(bar_id, 128, bad || need)) {
+                if (named_bar_any(bar_id, NBAR, bad || need)) {
                     {
                         float wm[NHW];
 #pragma unroll
-                        for (int h = 0; h < NHW; ++h) {
-                            wm[h] = x[0][h];
-#pragma unroll
-                            for (int hf = 1; hf < RT; ++hf) wm[h] = fmaxf(wm[h], x[hf][h]);
-                        }
+                        for (int h = 0; h < NHW; ++h) wm[h] = x[h];
                         warp_max_transpose8<NHW, C::LOG2NHW>(wm, lane);
                         if (lane < NHW)
-                            reinterpret_cast<float *>(&sm->wmax[wgi][j2][q4][0])[transpose_head8<NHW, C::LOG2NHW>(lane)] = wm[0];
+                            reinterpret_cast<float *>(&sm->wmax[wg][j2][wq][0])[transpose_head8<NHW, C::LOG2NHW>(lane)] = wm[0];
                     }
-                    if (named_bar_any(bar_id, 128, bad)) {
-                        bad = true;
-                        if constexpr (PP == 1) {
-                            ok = false;
-                            break;
-                        } else {
-                            continue;  // skip to the unit's merge barrier
-                        }
+                    if (named_bar_any(bar_id, NBAR, bad)) {
+                        ok = false;
+                        break;
                     }
 #pragma unroll
                     for (int h4 = 0; h4 < C::NHW4; ++h4) {
-                        const float4 a = sm->wmax[wgi][j2][0][h4], b = sm->wmax[wgi][j2][1][h4];
-                        const float4 c = sm->wmax[wgi][j2][2][h4], e = sm->wmax[wgi][j2][3][h4];
-                        const float t4[4] = {fmaxf(fmaxf(a.x, b.x), fmaxf(c.x, e.x)),
-                                             fmaxf(fmaxf(a.y, b.y), fmaxf(c.y, e.y)),
-                                             fmaxf(fmaxf(a.z, b.z), fmaxf(c.z, e.z)),
-                                             fmaxf(fmaxf(a.w, b.w), fmaxf(c.w, e.w))};
+                        float4 a = sm->wmax[wg][j2][0][h4];
+#pragma unroll
+                        for (int q = 1; q < 4 * RS; ++q) {
+                            const float4 b = sm->wmax[wg][j2][q][h4];
+                            a.x = fmaxf(a.x, b.x);
+                            a.y = fmaxf(a.y, b.y);
+                            a.z = fmaxf(a.z, b.z);
+                            a.w = fmaxf(a.w, b.w);
+                        }
+                        const float t4[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
                         for (int e4 = 0; e4 < 4; ++e4) {
                             const int h = h4 * 4 + e4;
@@ -681,25 +668,15 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                     for (int h = 0; h < NHW; ++h) alpha[h] = 1.f;
                 }
 
-                // P buffer j2 last fed the PV of this warpgroup's previous tile.  With one
-                // warpgroup that PV is known complete (its O was folded during the tile in
-                // between); with two, wait for it here, or P could be overwritten under a running
-                // PV and p_full[j2] could run a phase ahead of the issuer.
-                if (PP == 2 && prev_t >= 0 && !bad &&
-                    !wait_bounded(&sm->o_full[prev_t % C::OB], (prev_t / C::OB) & 1, abort_flag, budget))
-                    bad = true;
-                // P of this thread's rows, as three e4m3 terms, one 16-byte chunk per term and
-                // row (the warpgroup's 16 heads; zero bytes for padding heads).
-#pragma unroll
-                for (int h = 0; h < NHW; ++h) l[h] *= alpha[h];
-#pragma unroll
-                for (int hf = 0; hf < RT; ++hf) {
+                // P of this thread's row, as three e4m3 terms, one 16-byte chunk per term (the
+                // group's 16 heads; zero bytes for padding heads).
+                {
                     float pv[16];
 #pragma unroll
                     for (int h = 0; h < 16; ++h) {
                         if (h < NHW) {
-                            pv[h] = x[hf][h] == -INFINITY ? 0.f : ex2_approx(x[hf][h] - m_run[h]);
-                            l[h] += pv[h];
+                            pv[h] = x[h] == -INFINITY ? 0.f : ex2_approx(x[h] - m_run[h]);
+                            l[h] = l[h] * alpha[h] + pv[h];
                         } else {
                             pv[h] = 0.f;
                         }
@@ -718,9 +695,7 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                             tw[0][k / 4] = tw[1][k / 4] = tw[2][k / 4] = 0u;
                         }
                     }
-                    const int trow = hf * 128 + row;
-                    const uint32_t off = p_chunk<RP>(trow, hbase >> 4);
-                    uint8_t *pt = p_base + j2 * C::P_BYTES + off;
+                    uint8_t *pt = p_base + j2 * C::P_BYTES + p_chunk<RP>(trow, hbase >> 4);
 #pragma unroll
                     for (int term = 0; term < 3; ++term)
                         *reinterpret_cast<uint4 *>(pt + term * C::P_TERM) = make_uint4(tw[term][0], tw[term][1], tw[term][2], tw[term][3]);
@@ -729,64 +704,30 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm->p_full[j2]);
 
-                // O of this warpgroup's previous tile was computed against the previous
-                // maximum; fold it in and move the sum to the current one.
-                if (prev_t >= 0 && !fold_o(prev_t, alpha)) bad = true;
-                prev_t = i;
+                // O(i-1) was computed against the previous maximum; fold it in and move the
+                // sum to the current one.
+                if (folds && jj > 0 && !fold_o(i - 1, alpha)) bad = true;
             }
             if (!ok) break;
-            if (prev_t >= 0 && (bad || !fold_o(prev_t, nullptr))) bad = true;
+            if (folds && (bad || !fold_o(i - 1, nullptr))) bad = true;
 #pragma unroll
             for (int h = 0; h < NHW; ++h) {
                 const float sum = warp_sum_f32(l[h]);
-                if (lane == 0) sm->lsum[wgi][q4][h] = sum;
+                if (lane == 0) sm->lsum[wg][wq][h] = sum;
             }
-            float Lh[NHW];
-            if constexpr (PP == 2) {
-                // The odd-tile warpgroup hands (O, m) to the even one through its own P buffer
-                // (free: its PVs are done); l went through lsum.
-                float *xo = reinterpret_cast<float *>(p_base + C::P_BYTES);
-                if (pp == 1) {
-                    if (dcol >= 0) {
-#pragma unroll
-                        for (int h = 0; h < NHW; ++h) xo[h * D + dcol] = O[h];
-                    }
-                    if (sm_tid < NHW) {
-                        float mv = -INFINITY;
-#pragma unroll
-                        for (int hh = 0; hh < NHW; ++hh)
-                            if (hh == sm_tid) mv = m_run[hh];
-                        sm->mx[sm_tid] = mv;
-                    }
-                }
-                if (named_bar_any(bar_pair, 256, bad)) {
-                    ok = false;
-                    break;
-                }
-                if (pp == 0) {
-#pragma unroll
-                    for (int h = 0; h < NHW; ++h) {
-                        const float m1 = sm->mx[h];
-                        const float L0 = sm->lsum[0][0][h] + sm->lsum[0][1][h] + sm->lsum[0][2][h] + sm->lsum[0][3][h];
-                        const float L1 = sm->lsum[1][0][h] + sm->lsum[1][1][h] + sm->lsum[1][2][h] + sm->lsum[1][3][h];
-                        const float M = fmaxf(m_run[h], m1);
-                        const float a0 = m_run[h] == -INFINITY ? 0.f : ex2_approx(m_run[h] - M);
-                        const float a1 = m1 == -INFINITY ? 0.f : ex2_approx(m1 - M);
-                        if (dcol >= 0) O[h] = O[h] * a0 + xo[h * D + dcol] * a1;
-                        Lh[h] = L0 * a0 + L1 * a1;
-                        m_run[h] = M;
-                    }
-                }
-            } else {
-                if (named_bar_any(bar_id, 128, bad)) {
-                    ok = false;
-                    break;
-                }
-#pragma unroll
-                for (int h = 0; h < NHW; ++h)
-                    Lh[h] = sm->lsum[wg][0][h] + sm->lsum[wg][1][h] + sm->lsum[wg][2][h] + sm->lsum[wg][3][h];
+            if (named_bar_any(bar_id, NBAR, bad)) {
+                ok = false;
+                break;
             }
-            if (pp == 0 && dcol >= 0) {
+            if (folds && dcol >= 0) {
+                float Lh[NHW];
+#pragma unroll
+                for (int h = 0; h < NHW; ++h) {
+                    float L = 0.f;
+#pragma unroll
+                    for (int q = 0; q < 4 * RS; ++q) L += sm->lsum[wg][q][h];
+                    Lh[h] = L;
+                }
                 if (sg.whole) {
 #pragma unroll
                     for (int h = 0; h < NHW; ++h) {
@@ -812,10 +753,8 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                     }
                 }
             }
-            // the next unit rewrites lsum (and the hand-over area) only after every thread
-            // has read it
-            if constexpr (PP == 2) named_bar_sync(bar_pair, 256);
-            else named_bar_sync(bar_id, 128);
+            // the next unit rewrites lsum only after every thread has read it
+            named_bar_sync(bar_id, NBAR);
         }
         if (!ok) fail();
     }
