@@ -34,6 +34,7 @@ METRIC = "GQA decode: achieved KV-read HBM GB/s (% of B200 peak); µs per decode
 DEFAULT_WORKLOAD = "llama2_70b_layer"
 PROFILE_DIR = os.path.join(ROOT, "profiles")
 SPLIT_KERNEL_SOURCES = ["decode_tc.cu", "device.cuh", "schedule.cuh"]
+SPLIT8_KERNEL_SOURCES = ("decode_tc8.cu", "device.cuh", "schedule.cuh")
 
 
 def parse():
@@ -78,23 +79,25 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
-def split_kernel_hash() -> str:
+def split_kernel_hash(sources=None) -> str:
     h = hashlib.sha256()
-    for name in SPLIT_KERNEL_SOURCES:
+    for name in sources or SPLIT_KERNEL_SOURCES:
         with open(os.path.join(ROOT, "grouped_query_attention_decode_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str):
+def profiled_traffic(workload: str, fp8: bool = False):
     """dram bytes per launch of the split kernel from a committed ncu summary, when it was taken
     on the current kernel source; else None."""
-    p = os.path.join(PROFILE_DIR, f"split_tc_{workload}.json")
+    stem = "split_tc8" if fp8 else "split_tc"
+    p = os.path.join(PROFILE_DIR, f"{stem}_{workload}.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
-    if d.get("kernel_source_hash") != split_kernel_hash():
+    sources = SPLIT8_KERNEL_SOURCES if fp8 else SPLIT_KERNEL_SOURCES
+    if d.get("kernel_source_hash") != split_kernel_hash(sources):
         return None
     return d.get("dram_bytes_per_launch_full_size")
 
@@ -366,7 +369,7 @@ def bench_ours(args, rank, world, local):
                 "achieved": round(achieved, 1),
                 "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                 "frac": round(achieved / peak, 4),
-                "traffic": profiled_traffic(w.name),
+                "traffic": profiled_traffic(w.name, w.fp8),
                 "algorithmic_bytes_per_launch": ideal,
                 "avg_launch_us": round(split_avg * 1e3, 3),
                 "launches_timed": len(split_ms),

@@ -443,6 +443,27 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             uint32_t idle_polls = 0;
             while (qk_more || pv_t < qk_t) {
                 bool progress = false;
+                // P.V first: it is what releases a stage, so it never waits behind the next
+                // tile's S^T.
+                if (pv_t < qk_t) {
+                    const int j2 = pv_t & 1;
+                    const int ob = pv_t % C::OB;
+                    if (mbar_test_wait(&sm->p_full[j2], (pv_t >> 1) & 1) &&
+                        (pv_t < C::OB || mbar_test_wait(&sm->o_empty[ob], ((pv_t / C::OB) - 1) & 1))) {
+                        tc_fence_after_sync();
+                        const uint64_t dv = desc_add8(dv0, (pv_t % S) * C::STAGE_BYTES);
+                        const uint64_t dp = desc_add8(dp0, j2 * C::P_BYTES);
+#pragma unroll
+                        for (int kk = 0; kk < T / 32; ++kk) {
+                            umma_f8(tmem + C::O_COL + ob * 3 * RP, desc_add8(dv, kk * 32 * ROWB),
+                                    desc_add8(dp, kk * 32 * RP), C::IDESC_PV, kk > 0 ? 1u : 0u);
+                        }
+                        umma_commit(&sm->o_full[ob]);
+                        umma_commit(&sm->kv_empty[pv_t % S]);
+                        ++pv_t;
+                        progress = true;
+                    }
+                }
                 if (qk_more) {
                     const int qb = sidx % C::QB;
                     if (!q_ready) q_ready = mbar_test_wait(&sm->q_full[qb], (sidx / C::QB) & 1);
@@ -470,25 +491,6 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                             q_ready = false;
                             qk_more = w.next(sg);
                         }
-                        progress = true;
-                    }
-                }
-                if (pv_t < qk_t) {
-                    const int j2 = pv_t & 1;
-                    const int ob = pv_t % C::OB;
-                    if (mbar_test_wait(&sm->p_full[j2], (pv_t >> 1) & 1) &&
-                        (pv_t < C::OB || mbar_test_wait(&sm->o_empty[ob], ((pv_t / C::OB) - 1) & 1))) {
-                        tc_fence_after_sync();
-                        const uint64_t dv = desc_add8(dv0, (pv_t % S) * C::STAGE_BYTES);
-                        const uint64_t dp = desc_add8(dp0, j2 * C::P_BYTES);
-#pragma unroll
-                        for (int kk = 0; kk < T / 32; ++kk) {
-                            umma_f8(tmem + C::O_COL + ob * 3 * RP, desc_add8(dv, kk * 32 * ROWB),
-                                    desc_add8(dp, kk * 32 * RP), C::IDESC_PV, kk > 0 ? 1u : 0u);
-                        }
-                        umma_commit(&sm->o_full[ob]);
-                        umma_commit(&sm->kv_empty[pv_t % S]);
-                        ++pv_t;
                         progress = true;
                     }
                 }
