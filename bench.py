@@ -189,7 +189,7 @@ def bench_ours(args, rank, world, local):
     if w.queries > 1:
         nws = gqa.load_library().gqa_decode_multi_workspace_size(w.B, w.queries, w.H_q, w.H_kv, w.d,
                                                                  gqa.DTYPE_BF16 if w.dtype == torch.bfloat16 else gqa.DTYPE_F32)
-        ws = torch.empty(nws, dtype=torch.uint8, device=dev)
+        ws = torch.zeros(nws, dtype=torch.uint8, device=dev)
     elif w.fp8:
         ws = gqa.alloc_workspace_fp8(w.B, w.H_q, w.H_kv, w.d, device=dev)
     else:

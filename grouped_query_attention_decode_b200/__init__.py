@@ -154,7 +154,7 @@ def alloc_workspace(B: int, H_q: int, H_kv: int, d: int, dtype: torch.dtype, dev
     n = workspace_size(B, H_q, H_kv, d, dtype)
     if n == 0:
         raise GQAError(-9, "no usable sm_100 device is current, or invalid sizes")
-    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
 
 
 def decode(q, k_cache, v_cache, seq_lens, scale: float, out=None, workspace=None, status=None,
@@ -238,7 +238,7 @@ def decode_multi(q, k_cache, v_cache, seq_lens, scale: float, out=None, workspac
         n = int(lib.gqa_decode_multi_workspace_size(B, Q, H_q, H_kv, d, _DTYPES[k_cache.dtype]))
         if n == 0:
             raise GQAError(-9, "no usable sm_100 device is current, or invalid sizes")
-        workspace = torch.empty(n, dtype=torch.uint8, device=q.device)
+        workspace = torch.zeros(n, dtype=torch.uint8, device=q.device)
     _check(lib.gqa_decode_multi(
         _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens), B, Q, H_q, H_kv, d, L_max,
         float(scale), _dtype(k_cache), _ptr(out), _ptr(workspace), workspace.numel(),
@@ -296,7 +296,7 @@ def alloc_workspace_fp8(B: int, H_q: int, H_kv: int, d: int, device=None):
     n = int(load_library().gqa_decode_workspace_size(B, H_q, H_kv, d, DTYPE_E4M3))
     if n == 0:
         raise GQAError(-9, "no usable sm_100 device is current, or invalid sizes")
-    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
 
 
 def kv_append_fp8(k_new, v_new, k_cache, v_cache, k_scale, v_scale, seq_lens, status=None,

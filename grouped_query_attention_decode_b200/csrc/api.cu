@@ -50,7 +50,7 @@ int current_sm_count(int *dev_out) {
 
 struct Geometry {
     int r, rb, RB, HB, UB;
-    long long units, slots, slot_floats, hdr_floats;
+    long long units, slots, slot_floats, hdr_floats, cnt_floats;
     size_t bytes;
 };
 
@@ -65,8 +65,12 @@ Geometry geometry(int B, int H_q, int H_kv, int d, int G, int Q = 1) {
     g.UB = H_kv * g.HB;
     g.units = static_cast<long long>(B) * g.UB;
     g.slots = G + g.units - 1;
-    g.slot_floats = static_cast<long long>(g.RB) * (d + 2);
-    g.hdr_floats = ((static_cast<long long>(B) + 1) * 8 + 255) / 256 * 64;  // 256-byte multiple
+    // O [RB][d], m [RB], l [RB], rounded up to whole 16-byte vectors (the merge reads o with
+    // 16-byte loads)
+    g.slot_floats = (static_cast<long long>(g.RB) * (d + 2) + 3) / 4 * 4;
+    // int64 header [B + 1], then the per-unit piece counters, each region a 256-byte multiple
+    g.cnt_floats = ((static_cast<long long>(B) + 1) * 8 + 255) / 256 * 64;
+    g.hdr_floats = g.cnt_floats + (g.units * kPieceGroups * 4 + 255) / 256 * 64;
     g.bytes = static_cast<size_t>((g.hdr_floats + g.slots * g.slot_floats) * 4 + 255) / 256 * 256;
     return g;
 }
@@ -206,6 +210,16 @@ extern "C" size_t gqa_decode_multi_workspace_size(int B, int Q, int H_q, int H_k
     return geometry(B, H_q, H_kv, d, sms, Q).bytes;
 }
 
+size_t gqa::decode_counter_region(int B, int H_q, int H_kv, int d, size_t *offset) {
+    if (check_shape(B, H_q, H_kv, d, 1, GQA_DTYPE_BF16) != GQA_OK) return 0;
+    int dev = 0;
+    const int sms = current_sm_count(&dev);
+    if (sms <= 0) return 0;
+    const Geometry g = geometry(B, H_q, H_kv, d, sms);
+    *offset = static_cast<size_t>(g.cnt_floats) * 4;
+    return static_cast<size_t>(g.hdr_floats - g.cnt_floats) * 4;
+}
+
 extern "C" size_t gqa_decode_workspace_size(int B, int H_q, int H_kv, int d, gqa_dtype_t dtype) {
     if (check_shape(B, H_q, H_kv, d, 1, dtype, true) != GQA_OK) return 0;
     int dev = 0;
@@ -244,6 +258,7 @@ int decode_impl(const void *q, const void *k_cache, const void *v_cache, const i
     if (Q < 1 || Q > 64) return GQA_ERR_SHAPE;
     const Geometry g = geometry(B, H_q, H_kv, d, sms, Q);
     if (workspace_bytes < g.bytes) return GQA_ERR_WORKSPACE;
+    if (g.slot_floats % 4 != 0 || g.hdr_floats % 4 != 0) return GQA_ERR_SHAPE;  // 16-byte slot vectors
 
     DecodeParams p;
     p.seq_lens = seq_lens;
@@ -279,6 +294,7 @@ int decode_impl(const void *q, const void *k_cache, const void *v_cache, const i
     p.wait_ns = g_wait_ns.load();
     p.slot_floats = g.slot_floats;
     p.hdr_floats = g.hdr_floats;
+    p.cnt = reinterpret_cast<int32_t *>(static_cast<float *>(workspace) + g.cnt_floats);
 
     cudaEvent_t ev0 = g_ev_before.load(), ev1 = g_ev_after.load();
     const bool profile = ev0 != nullptr && ev1 != nullptr;
@@ -320,7 +336,7 @@ int decode_impl(const void *q, const void *k_cache, const void *v_cache, const i
     }
     if (res != GQA_OK) return res;
     if (profile && cudaEventRecord(ev1, stream) != cudaSuccess) return GQA_ERR_CUDA;
-    return launch_combine(p, stream);
+    return GQA_OK;
 }
 
 }  // namespace

@@ -37,7 +37,9 @@ split_f32_kernel(const float *__restrict__ q, const float *__restrict__ kc,
     float *const ms = ss + C::RBMAX * T;                 // running max per head (log2 units)
     float *const as = ms + C::RBMAX;                     // rescale factor of the last tile
     float *const ls = as + C::RBMAX;                     // running softmax denominator
-    __shared__ long long s_begin, s_end, s_off0;
+    __shared__ long long s_begin, s_end, s_off0, s_total;
+    __shared__ int s_flag;
+    __shared__ PendingPiece s_pend[2];
     __shared__ int s_b0;
 
     const int tid = threadIdx.x;
@@ -53,6 +55,7 @@ split_f32_kernel(const float *__restrict__ q, const float *__restrict__ kc,
             s_end = cr.end;
             s_b0 = cr.b0;
             s_off0 = cr.off0;
+            s_total = cr.total;
         }
     }
     __syncthreads();
@@ -63,10 +66,11 @@ split_f32_kernel(const float *__restrict__ q, const float *__restrict__ kc,
     cr.end = s_end;
     cr.b0 = s_b0;
     cr.off0 = s_off0;
-    cr.total = 0;
+    cr.total = s_total;
     SegmentWalker w;
     w.init(p, cr);
     Segment sg;
+    PieceTickets tickets;
     constexpr int ACC = C::RBMAX * D / 256;
     while (w.next(sg)) {
         // columns of the unit: (token j, head h') pairs, j * rb + h'
@@ -186,7 +190,11 @@ split_f32_kernel(const float *__restrict__ q, const float *__restrict__ kc,
             }
         }
         __syncthreads();
+        if (!sg.whole) tickets.record(p, sg, 0, tid, s_pend);
     }
+    // units cut into pieces are merged by the CTA holding the last ticket
+    tickets.finish(p, cr.total, 0, 0, p.RB, tid, 256, s_pend, &s_flag, [] { __syncthreads(); });
+    zero_empty_units(p, blockIdx.x, tid, 256);
 }
 
 template <int D>

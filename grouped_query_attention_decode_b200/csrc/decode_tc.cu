@@ -72,7 +72,9 @@ struct TcCfg {
         int abort;
         int b0;
         int pad_;
-        long long begin, end, off0;
+        long long begin, end, off0, total;
+        int pflag[kPieceGroups];
+        PendingPiece pend[kPieceGroups][2];
         float4 wmax[NWG][2][4][NHW4];  // per group, tile parity, warp: per-head warp maxima
         float lsum[NWG][4][NHW];
     };
@@ -191,6 +193,7 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             sm->end = cr.end;
             sm->b0 = cr.b0;
             sm->off0 = cr.off0;
+            sm->total = cr.total;
         }
     }
     tc_fence_before_sync();
@@ -204,7 +207,7 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     cr.end = sm->end;
     cr.b0 = sm->b0;
     cr.off0 = sm->off0;
-    cr.total = 0;
+    cr.total = sm->total;
     volatile int *abort_flag = &sm->abort;
     const uint64_t budget = p.wait_ns;
 
@@ -435,6 +438,7 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         int i = 0;
         bool ok = true;
         float O[NHW], l[NHW], m_run[NHW], alpha[NHW];
+        PieceTickets tickets;
         while (ok && w.next(sg)) {
 #pragma unroll
             for (int h = 0; h < NHW; ++h) {
@@ -656,10 +660,19 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     }
                 }
             }
-            // the next piece rewrites lsum only after every thread has read it
+            // the next piece rewrites lsum only after every thread has read it (and the slot
+            // stores are ordered before the ticket)
             named_bar_sync(bar_id, 128);
+            if (!sg.whole) tickets.record(p, sg, wg, sm_tid - 128 * wg, sm->pend[wg]);
         }
-        if (!ok) fail();
+        if (!ok) {
+            fail();
+        } else {
+            // units cut into pieces are merged by the CTA holding the last ticket
+            tickets.finish(p, cr.total, wg, hbase, hbase + NHW, sm_tid - 128 * wg, 128, sm->pend[wg],
+                           &sm->pflag[wg], [&] { named_bar_sync(bar_id, 128); });
+            zero_empty_units(p, blockIdx.x, sm_tid, 128 * C::NWG);
+        }
     }
 
     tc_fence_before_sync();

@@ -85,7 +85,9 @@ struct Tc8Cfg {
         int abort;
         int b0;
         int pad_;
-        long long begin, end, off0;
+        long long begin, end, off0, total;
+        int pflag[kPieceGroups];
+        PendingPiece pend[kPieceGroups][2];
         float qf[2][RP];                    // score factor of each column: scale * k_scale / c_h
         float vsc[2];                       // v_scale of the unit's key/value head
         float4 wmax[NWG][2][4 * RS][NHW4];  // per head slice, S buffer, warp: warp maxima
@@ -228,6 +230,7 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             sm->end = cr.end;
             sm->b0 = cr.b0;
             sm->off0 = cr.off0;
+            sm->total = cr.total;
         }
     }
     tc_fence_before_sync();
@@ -241,7 +244,7 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     cr.end = sm->end;
     cr.b0 = sm->b0;
     cr.off0 = sm->off0;
-    cr.total = 0;
+    cr.total = sm->total;
     volatile int *abort_flag = &sm->abort;
     const uint64_t budget = p.wait_ns;
 
@@ -538,6 +541,7 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         int i = 0, sidx = 0;
         bool ok = true;
         float O[NHW], l[NHW], m_run[NHW], alpha[NHW], f[NHW];
+        PieceTickets tickets;
         // O of tile t folded into the running sum, scaled by `scale_by` (first row half only)
         auto fold_o = [&](int t, const float *scale_by) -> bool {
             const int ob = t % C::OB;
@@ -755,10 +759,19 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                     }
                 }
             }
-            // the next unit rewrites lsum only after every thread has read it
+            // the next unit rewrites lsum only after every thread has read it (and the slot
+            // stores are ordered before the ticket)
             named_bar_sync(bar_id, NBAR);
+            if (!sg.whole) tickets.record(p, sg, wg, sm_tid, sm->pend[wg]);
         }
-        if (!ok) fail();
+        if (!ok) {
+            fail();
+        } else {
+            // units cut into pieces are merged by the CTA holding the last ticket
+            tickets.finish(p, cr.total, wg, hbase, hbase + NHW, sm_tid, NBAR, sm->pend[wg], &sm->pflag[wg],
+                           [&] { named_bar_sync(bar_id, NBAR); });
+            zero_empty_units(p, blockIdx.x, threadIdx.x - 64, 128 * C::NSW);
+        }
     }
 
     tc_fence_before_sync();

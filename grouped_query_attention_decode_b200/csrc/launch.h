@@ -20,10 +20,12 @@ int launch_split_tc(const TmaMaps &maps, const DecodeParams &p, cudaStream_t str
 int tc_q_box_rows(int heads_per_unit);
 int launch_split_f32(const DecodeParams &p, const float *q, const float *kc, const float *vc,
                      cudaStream_t stream);
-int launch_combine(const DecodeParams &p, cudaStream_t stream);
 // FP8 (e4m3) cache: the split kernel (K/V maps of uint8 codes with box rows tc8_tile_rows or
 // the page size, and 8-row boxes; q is read from global memory) and the quantising append.
 int tc8_tile_rows(int heads_per_unit);
+// Byte offset and size of the per-unit piece counters inside a decode workspace for these
+// sizes on the current device (0 bytes when the sizes are invalid).
+size_t decode_counter_region(int B, int H_q, int H_kv, int d, size_t *offset);
 int launch_split_tc8(const TmaMaps &maps, const void *q, const DecodeParams &p, cudaStream_t stream);
 int launch_append_fp8(const void *k_new, const void *v_new, bool bf16_in, void *k_cache,
                       void *v_cache, const float *k_scale, const float *v_scale, int32_t *seq_lens,

@@ -15,6 +15,7 @@
 #include <mutex>
 
 #include "gqa.h"
+#include "launch.h"
 
 namespace {
 
@@ -65,6 +66,12 @@ extern "C" int gqa_decode_noalloc(const void *q, const void *k_cache, const void
     void *ws = nullptr;
     const int rc = scratch_address(&ws);
     if (rc != GQA_OK) return rc;
+    // The workspace's piece counters must be zero; a call that timed out may have left some
+    // set, and the caller cannot reach this array, so clear them on the stream every time.
+    size_t off = 0;
+    const size_t cnt_bytes = gqa::decode_counter_region(B, H_q, H_kv, d, &off);
+    if (cnt_bytes > 0 && cudaMemsetAsync(static_cast<unsigned char *>(ws) + off, 0, cnt_bytes, stream) != cudaSuccess)
+        return GQA_ERR_CUDA;
     return gqa_decode(q, k_cache, v_cache, seq_lens, B, H_q, H_kv, d, L_max, scale, dtype, out,
                       ws, kScratchBytes, status, stream);
 }

@@ -44,9 +44,10 @@ struct DecodeParams {
     // FP8 (e4m3) cache: a code of key/value head g stands for value(code) * k_scale[g] (K)
     // or value(code) * v_scale[g] (V); nullptr for 16- and 32-bit caches.
     const float *k_scale, *v_scale;
+    int32_t *cnt;                     // [units] pieces of each unit finished in this call (0 between calls)
     float scale_log2;                 // softmax scale * log2(e)
     unsigned long long wait_ns;       // bound of every pipeline wait
-    long long slot_floats;            // RB * (d + 2)
+    long long slot_floats;            // RB * (d + 2) rounded up to a multiple of 4
     long long hdr_floats;             // header length in floats (int64 offsets [B + 1])
 };
 
@@ -156,6 +157,8 @@ struct Segment {
     int first;       // first attended row (0 unless a sliding window cuts the front)
     int unit;        // unit index b * UB + (kvh * HB + hb)
     bool whole;      // the piece is the entire unit
+    int nt;          // tiles of the unit
+    long long uoff;  // line position of the unit's first tile
 };
 
 // Walks the segments of one CTA range in order.  Each role of the CTA runs its own walker;
@@ -212,11 +215,165 @@ struct SegmentWalker {
         s.n = n;
         s.first = first_row(n, window);
         s.unit = b * UB + k;
+        s.nt = nt;
+        s.uoff = off + static_cast<long long>(k) * nt;
         s.whole = (j0 == 0 && len == nt);
         t += len;
         return true;
     }
 };
+
+// ---------------------------------------------------------------------- piece merge
+// A unit cut into several pieces (by CTA ranges) is merged by the CTA that finishes its last
+// piece: every piece stores its partial (o, m, l) in its slot, fences it, and takes a ticket
+// from the unit's counter; the CTA holding the last ticket merges all slots -- the log-sum-exp
+// combine below -- writes the unit's output and puts the counter back to zero.
+//
+// A piece c of a unit holds, per column, the unnormalised sum o_c = sum_t 2^(x_t - m_c) v_t,
+// its reference m_c (log2 units) and l_c = sum_t 2^(x_t - m_c).  Softmax is a ratio of sums of
+// exponentials, so the pieces merge exactly:
+//     M = max_c m_c,   out = sum_c 2^(m_c - M) o_c / sum_c 2^(m_c - M) l_c.
+// The pages state the blockwise idea (split a long sequence into blocks, compute them
+// independently, merge: "GQA注意力机制", section 4.2); the merge rule is this softmax algebra.
+
+// CTAs in [c0, c1] whose ranges hold tiles of the unit at [uoff, uoff + nt); with fewer tiles
+// than CTAs some ranges are empty and hold no piece.
+__device__ __forceinline__ int unit_pieces(long long uoff, int nt, long long total, int G, int &c0,
+                                           int &c1) {
+    c0 = static_cast<int>(cta_of_tile(uoff, total, G));
+    c1 = static_cast<int>(cta_of_tile(uoff + nt - 1, total, G));
+    if (total >= G) return c1 - c0 + 1;
+    int np = 0;
+    for (int c = c0; c <= c1; ++c) np += cta_range_begin(c, total, G) < cta_range_begin(c + 1, total, G);
+    return np;
+}
+
+// Counters per unit: one per group of threads that writes (and merges) its own columns.
+constexpr int kPieceGroups = 4;
+
+// A piece whose ticket was taken; only the first and the last segment of a CTA range can be
+// partial pieces, so a CTA has at most two.
+struct PendingPiece {
+    long long uoff;
+    int unit, b, kvh, hb, nt;
+};
+
+// Ticket for this group's columns of `unit`: atomic add with release semantics (the group's
+// slot stores, ordered before it by the group barrier the caller just passed, become visible
+// at GPU scope first) and acquire semantics (a last piece then sees every other slot).  The
+// returned count is the number of pieces that finished before this one.
+__device__ __forceinline__ int take_ticket(const DecodeParams &p, int unit, int group) {
+    int old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;"
+                 : "=r"(old)
+                 : "l"(p.cnt + static_cast<long long>(unit) * kPieceGroups + group)
+                 : "memory");
+    return old;
+}
+
+// The group (threads tid < nthr) that took a unit's last ticket merges that unit's columns
+// [h0, h1): a one-pass log-sum-exp over the pieces' slots, four outputs per step, and puts the
+// counter back to zero.
+__device__ inline void merge_unit(const DecodeParams &p, const PendingPiece &u, long long total,
+                                  int group, int h0, int h1, int tid, int nthr) {
+    int c0, c1;
+    unit_pieces(u.uoff, u.nt, total, p.G, c0, c1);
+    const int nh = p.RB, d = p.d;
+    h1 = min(h1, nh);
+    const float *base = p.ws + p.hdr_floats + static_cast<long long>(u.unit) * p.slot_floats;
+    const bool some_empty = total < p.G;
+    const int nvec = (h1 - h0) * d / 4;
+    // four vectors per thread per round, all loaded before any store
+    for (int v0 = tid; v0 < nvec; v0 += 4 * nthr) {
+        float4 res[4];
+        long long dst[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int v = v0 + j * nthr;
+            dst[j] = -1;
+            res[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (v >= nvec) continue;
+            const int idx = h0 * d + 4 * v;
+            const int h = idx / d;
+            const long long orow = out_row(p, u.b, u.kvh, u.hb, h);
+            if (orow < 0) continue;
+            float M = -INFINITY, den = 0.f;
+            float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int c = c0; c <= c1; ++c) {
+                if (some_empty && cta_range_begin(c, total, p.G) >= cta_range_begin(c + 1, total, p.G)) continue;
+                const float *sl = base + static_cast<long long>(c) * p.slot_floats;
+                const float m = __ldcg(sl + nh * d + h);
+                const float l = __ldcg(sl + nh * d + nh + h);
+                const float4 o = __ldcg(reinterpret_cast<const float4 *>(sl + idx));
+                if (m == -INFINITY) continue;
+                if (m > M) {
+                    const float sc = M == -INFINITY ? 0.f : ex2_approx(M - m);
+                    num.x *= sc; num.y *= sc; num.z *= sc; num.w *= sc;
+                    den *= sc;
+                    M = m;
+                }
+                const float wgt = ex2_approx(m - M);
+                num.x = fmaf(wgt, o.x, num.x);
+                num.y = fmaf(wgt, o.y, num.y);
+                num.z = fmaf(wgt, o.z, num.z);
+                num.w = fmaf(wgt, o.w, num.w);
+                den = fmaf(wgt, l, den);
+            }
+            const float inv = 1.f / den;
+            res[j] = make_float4(num.x * inv, num.y * inv, num.z * inv, num.w * inv);
+            dst[j] = orow * d + (idx - h * d);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            if (dst[j] >= 0) *reinterpret_cast<float4 *>(p.out + dst[j]) = res[j];
+    }
+    if (tid == 0) p.cnt[static_cast<long long>(u.unit) * kPieceGroups + group] = 0;
+}
+
+// Bookkeeping of one group's partial pieces: record(...) right after the group barrier that
+// follows a partial piece's slot stores; finish(...) once, after the CTA's last segment.
+struct PieceTickets {
+    int n = 0;
+    int ticket[2] = {0, 0};
+
+    __device__ void record(const DecodeParams &p, const Segment &sg, int group, int tid, PendingPiece *pend) {
+        if (n < 2 && tid == 0) {
+            pend[n] = PendingPiece{sg.uoff, sg.unit, sg.b, sg.kvh, sg.hb, sg.nt};
+            ticket[n] = take_ticket(p, sg.unit, group);
+        }
+        ++n;
+    }
+
+    template <typename Bar>
+    __device__ void finish(const DecodeParams &p, long long total, int group, int h0, int h1, int tid, int nthr,
+                           PendingPiece *pend, int *flag, Bar bar) {
+        for (int k = 0; k < n && k < 2; ++k) {
+            if (tid == 0) {
+                int c0, c1;
+                *flag = ticket[k] == unit_pieces(pend[k].uoff, pend[k].nt, total, p.G, c0, c1) - 1;
+            }
+            bar();
+            if (*flag) merge_unit(p, pend[k], total, group, h0, h1, tid, nthr);
+            bar();
+        }
+    }
+};
+
+// Units with no rows (a sequence of length 0, or one refused as out of range) get zero
+// output; CTA `cta` of G covers units cta, cta + G, ...
+__device__ inline void zero_empty_units(const DecodeParams &p, int cta, int tid, int nthr) {
+    const int units = p.B * p.UB;
+    for (int u = cta; u < units; u += p.G) {
+        const int b = u / p.UB;
+        if (seq_tiles(valid_len(p.seq_lens[b], p.L_max, p.Q), p) != 0) continue;
+        const int k = u - b * p.UB;
+        const int kvh = k / p.HB, hb = k - kvh * p.HB;
+        for (int idx = tid; idx < p.RB * p.d; idx += nthr) {
+            const long long orow = out_row(p, b, kvh, hb, idx / p.d);
+            if (orow >= 0) p.out[orow * p.d + idx % p.d] = 0.f;
+        }
+    }
+}
 
 // Tiles ahead of the copy at which the paged producer loads page ids.
 constexpr int kPageAhead = 2;

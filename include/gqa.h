@@ -125,10 +125,13 @@ size_t gqa_decode_workspace_size(int B, int H_q, int H_kv, int d, gqa_dtype_t dt
  *   scale      softmax scale, usually 1/sqrt(d)
  *   out        [B][H_q][d] float32 device, written
  *   workspace  device scratch of at least gqa_decode_workspace_size() bytes, 256-byte aligned;
- *              owned by the caller, overwritten by every call.  Two gqa_decode calls that may
- *              run at the same time must not share one workspace.
+ *              owned by the caller.  It must be zero-filled once before its first use
+ *              (cudaMemset): it holds per-unit counters that every completed call leaves at
+ *              zero again.  After a call that reported GQA_STATUS_WAIT_TIMEOUT, zero it again.
+ *              Two calls that may run at the same time must not share one workspace.
  *   status     int32 device or NULL
- * Launches two kernels on `stream` (a split-KV pass and a log-sum-exp combine).
+ * Launches one kernel on `stream`: a split-KV pass whose CTAs merge the pieces of a split
+ * sequence themselves (log-sum-exp combine by the CTA that finishes the last piece).
  * Returns GQA_OK or a GQA_ERR_* code.
  */
 int gqa_decode(const void *q, const void *k_cache, const void *v_cache, const int32_t *seq_lens,
@@ -267,7 +270,9 @@ int gqa_decode_paged_fp8(const void *q, const void *k_pool, const void *v_pool,
  *     with GQA_ERR_SCRATCH_LIMIT before anything runs (use gqa_decode with a workspace).
  *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
  *     with that device current and caches it; make that first call before any stream capture.
- *   - Nothing in the array needs to start at zero: each call writes what it later reads.
+ *   - Each call first clears the array's counters with one cudaMemsetAsync on `stream` (the
+ *     zero start gqa_decode requires of a workspace), so a call that timed out leaves no
+ *     trace for the next one.
  *   - Every call shares the one array and it keeps the last call's contents.  Two calls that
  *     may overlap on the GPU (different streams, or different host threads without ordering)
  *     race on it and produce wrong results; order them on one stream.

@@ -44,7 +44,7 @@ def test_noalloc_matches_workspace_entry_point(w):
     ref = torch.empty((w.B, w.H_q, w.d), dtype=torch.float32, device=dev)
     nbytes = lib.gqa_decode_workspace_size(w.B, w.H_q, w.H_kv, w.d, dt)
     assert 0 < nbytes
-    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
     rc = lib.gqa_decode(_p(q), _p(kc), _p(vc), _p(lens), *args, _p(ref), _p(ws), nbytes,
                         _p(status), stream)
     assert rc == 0, gqa.status_string(rc)
