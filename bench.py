@@ -1,5 +1,5 @@
 #!/usr/bin/env python3
-"""Benchmark of one GQA decode step (KV append + split-KV decode + combine) on B200.
+"""Benchmark of one GQA decode step (KV append + split-KV decode with its in-kernel merge) on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
 
@@ -363,7 +363,7 @@ def bench_ours(args, rank, world, local):
                 "l2": "inputs larger than L2: two cache copies alternate between steps "
                       f"({2 * caches[0][0].numel() * 2 * w.elem_bytes / 1e6:.0f} MB)",
             },
-            "gpu_launches": 3 * K,
+            "gpu_launches": 2 * K,
             "roofline": {
                 "bound": "hbm", "kernel": "split_tc8_kernel" if w.fp8 else "split_tc_kernel",
                 "achieved": round(achieved, 1),
@@ -490,7 +490,7 @@ def profile_run(args, local):
     st = int(status.item())
     assert st == 0, f"device status {st}"
     return {"profile_run": w.name, "steps": args.steps, "warmup": args.warmup,
-            "launches_per_step": 3}
+            "launches_per_step": 2}
 
 
 def bench_reference(args, rank, world):
