@@ -71,6 +71,7 @@ split_f32_kernel(const float *__restrict__ q, const float *__restrict__ kc,
     w.init(p, cr);
     Segment sg;
     PieceTickets tickets;
+    zero_empty_units(p, blockIdx.x, tid, 256);  // units with no rows get zeros
     constexpr int ACC = C::RBMAX * D / 256;
     while (w.next(sg)) {
         // columns of the unit: (token j, head h') pairs, j * rb + h'
@@ -194,7 +195,6 @@ split_f32_kernel(const float *__restrict__ q, const float *__restrict__ kc,
     }
     // units cut into pieces are merged by the CTA holding the last ticket
     tickets.finish(p, cr.total, 0, 0, p.RB, tid, 256, s_pend, &s_flag, [] { __syncthreads(); });
-    zero_empty_units(p, blockIdx.x, tid, 256);
 }
 
 template <int D>

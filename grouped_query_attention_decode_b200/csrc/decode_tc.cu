@@ -439,6 +439,8 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         bool ok = true;
         float O[NHW], l[NHW], m_run[NHW], alpha[NHW];
         PieceTickets tickets;
+        // units with no rows get zeros (while the first tiles are still on their way)
+        zero_empty_units(p, blockIdx.x, sm_tid, 128 * C::NWG);
         while (ok && w.next(sg)) {
 #pragma unroll
             for (int h = 0; h < NHW; ++h) {
@@ -671,7 +673,6 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             // units cut into pieces are merged by the CTA holding the last ticket
             tickets.finish(p, cr.total, wg, hbase, hbase + NHW, sm_tid - 128 * wg, 128, sm->pend[wg],
                            &sm->pflag[wg], [&] { named_bar_sync(bar_id, 128); });
-            zero_empty_units(p, blockIdx.x, sm_tid, 128 * C::NWG);
         }
     }
 

@@ -542,6 +542,8 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         bool ok = true;
         float O[NHW], l[NHW], m_run[NHW], alpha[NHW], f[NHW];
         PieceTickets tickets;
+        // units with no rows get zeros (while the first tiles are still on their way)
+        zero_empty_units(p, blockIdx.x, threadIdx.x - 64, 128 * C::NSW);
         // O of tile t folded into the running sum, scaled by `scale_by` (first row half only)
         auto fold_o = [&](int t, const float *scale_by) -> bool {
             const int ob = t % C::OB;
@@ -770,7 +772,6 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             // units cut into pieces are merged by the CTA holding the last ticket
             tickets.finish(p, cr.total, wg, hbase, hbase + NHW, sm_tid, NBAR, sm->pend[wg], &sm->pflag[wg],
                            [&] { named_bar_sync(bar_id, NBAR); });
-            zero_empty_units(p, blockIdx.x, threadIdx.x - 64, 128 * C::NSW);
         }
     }
 
