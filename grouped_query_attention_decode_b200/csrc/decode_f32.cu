@@ -37,10 +37,10 @@ split_f32_kernel(const float *__restrict__ q, const float *__restrict__ kc,
     float *const ms = ss + C::RBMAX * T;                 // running max per head (log2 units)
     float *const as = ms + C::RBMAX;                     // rescale factor of the last tile
     float *const ls = as + C::RBMAX;                     // running softmax denominator
-    __shared__ long long s_begin, s_end, s_off0, s_total;
+    __shared__ long long s_begin, s_end, s_off0, s_offl, s_total;
     __shared__ int s_flag;
     __shared__ PendingPiece s_pend[2];
-    __shared__ int s_b0;
+    __shared__ int s_b0, s_bl;
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -55,6 +55,8 @@ split_f32_kernel(const float *__restrict__ q, const float *__restrict__ kc,
             s_end = cr.end;
             s_b0 = cr.b0;
             s_off0 = cr.off0;
+            s_bl = cr.bl;
+            s_offl = cr.offl;
             s_total = cr.total;
         }
     }
@@ -66,11 +68,14 @@ split_f32_kernel(const float *__restrict__ q, const float *__restrict__ kc,
     cr.end = s_end;
     cr.b0 = s_b0;
     cr.off0 = s_off0;
+    cr.bl = s_bl;
+    cr.offl = s_offl;
     cr.total = s_total;
     SegmentWalker w;
     w.init(p, cr);
     Segment sg;
     PieceTickets tickets;
+    int nseg = 0;
     zero_empty_units(p, blockIdx.x, tid, 256);  // units with no rows get zeros
     constexpr int ACC = C::RBMAX * D / 256;
     while (w.next(sg)) {
@@ -192,6 +197,8 @@ split_f32_kernel(const float *__restrict__ q, const float *__restrict__ kc,
         }
         __syncthreads();
         if (!sg.whole) tickets.record(p, sg, 0, tid, s_pend);
+        // the range's partial pieces come first: merge what they complete right away
+        if (++nseg == 2) tickets.finish(p, cr.total, 0, 0, p.RB, tid, 256, s_pend, &s_flag, [] { __syncthreads(); });
     }
     // units cut into pieces are merged by the CTA holding the last ticket
     tickets.finish(p, cr.total, 0, 0, p.RB, tid, 256, s_pend, &s_flag, [] { __syncthreads(); });

@@ -70,9 +70,8 @@ struct TcCfg {
         uint64_t mma_done;
         uint32_t tmem_base;
         int abort;
-        int b0;
-        int pad_;
-        long long begin, end, off0, total;
+        int b0, bl;
+        long long begin, end, off0, offl, total;
         int pflag[kPieceGroups];
         PendingPiece pend[kPieceGroups][2];
         float4 wmax[NWG][2][4][NHW4];  // per group, tile parity, warp: per-head warp maxima
@@ -193,6 +192,8 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             sm->end = cr.end;
             sm->b0 = cr.b0;
             sm->off0 = cr.off0;
+            sm->bl = cr.bl;
+            sm->offl = cr.offl;
             sm->total = cr.total;
         }
     }
@@ -207,6 +208,8 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     cr.end = sm->end;
     cr.b0 = sm->b0;
     cr.off0 = sm->off0;
+    cr.bl = sm->bl;
+    cr.offl = sm->offl;
     cr.total = sm->total;
     volatile int *abort_flag = &sm->abort;
     const uint64_t budget = p.wait_ns;
@@ -439,6 +442,7 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         bool ok = true;
         float O[NHW], l[NHW], m_run[NHW], alpha[NHW];
         PieceTickets tickets;
+        int nseg = 0;
         // units with no rows get zeros (while the first tiles are still on their way)
         zero_empty_units(p, blockIdx.x, sm_tid, 128 * C::NWG);
         while (ok && w.next(sg)) {
@@ -666,6 +670,10 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             // stores are ordered before the ticket)
             named_bar_sync(bar_id, 128);
             if (!sg.whole) tickets.record(p, sg, wg, sm_tid - 128 * wg, sm->pend[wg]);
+            // the range's partial pieces come first: merge what they complete right away
+            if (++nseg == 2)
+                tickets.finish(p, cr.total, wg, hbase, hbase + NHW, sm_tid - 128 * wg, 128, sm->pend[wg],
+                               &sm->pflag[wg], [&] { named_bar_sync(bar_id, 128); });
         }
         if (!ok) {
             fail();

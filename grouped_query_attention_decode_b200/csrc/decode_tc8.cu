@@ -83,9 +83,8 @@ struct Tc8Cfg {
         uint64_t mma_done;
         uint32_t tmem_base;
         int abort;
-        int b0;
-        int pad_;
-        long long begin, end, off0, total;
+        int b0, bl;
+        long long begin, end, off0, offl, total;
         int pflag[kPieceGroups];
         PendingPiece pend[kPieceGroups][2];
         float qf[2][RP];                    // score factor of each column: scale * k_scale / c_h
@@ -230,6 +229,8 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             sm->end = cr.end;
             sm->b0 = cr.b0;
             sm->off0 = cr.off0;
+            sm->bl = cr.bl;
+            sm->offl = cr.offl;
             sm->total = cr.total;
         }
     }
@@ -244,6 +245,8 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     cr.end = sm->end;
     cr.b0 = sm->b0;
     cr.off0 = sm->off0;
+    cr.bl = sm->bl;
+    cr.offl = sm->offl;
     cr.total = sm->total;
     volatile int *abort_flag = &sm->abort;
     const uint64_t budget = p.wait_ns;
@@ -542,6 +545,7 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         bool ok = true;
         float O[NHW], l[NHW], m_run[NHW], alpha[NHW], f[NHW];
         PieceTickets tickets;
+        int nseg = 0;
         // units with no rows get zeros (while the first tiles are still on their way)
         zero_empty_units(p, blockIdx.x, threadIdx.x - 64, 128 * C::NSW);
         // O of tile t folded into the running sum, scaled by `scale_by` (first row half only)
@@ -765,6 +769,10 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             // stores are ordered before the ticket)
             named_bar_sync(bar_id, NBAR);
             if (!sg.whole) tickets.record(p, sg, wg, sm_tid, sm->pend[wg]);
+            // the range's partial pieces come first: merge what they complete right away
+            if (++nseg == 2)
+                tickets.finish(p, cr.total, wg, hbase, hbase + NHW, sm_tid, NBAR, sm->pend[wg], &sm->pflag[wg],
+                               [&] { named_bar_sync(bar_id, NBAR); });
         }
         if (!ok) {
             fail();

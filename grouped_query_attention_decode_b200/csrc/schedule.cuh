@@ -100,6 +100,8 @@ struct CtaRange {
     long long begin, end, total;
     int b0;          // first sequence with a tile in [begin, end) (valid when begin < end)
     long long off0;  // first tile of sequence b0 on the line
+    int bl;          // sequence holding the range's last tile end - 1
+    long long offl;  // first tile of sequence bl on the line
 };
 
 // Whole warp: total tiles, this CTA's range and where it starts.  When `hdr` is not null the
@@ -128,20 +130,29 @@ __device__ inline CtaRange locate_cta_range(const DecodeParams &p, int cta, int 
     cr.end = cta_range_begin(cta + 1, run, p.G);
     cr.b0 = 0;
     cr.off0 = 0;
+    cr.bl = 0;
+    cr.offl = 0;
     if (cr.begin >= cr.end) return cr;
     long long off = 0;
+    bool found0 = false;
     for (int base = 0; base < p.B; base += 32) {
         const int b = base + lane;
         const int n = b < p.B ? valid_len(p.seq_lens[b], p.L_max, p.Q) : 0;
         const long long v = static_cast<long long>(seq_tiles(n, p)) * p.UB;
         const long long incl = warp_incl_scan(v, lane);
         const long long excl = incl - v;
-        const bool hit = v > 0 && off + excl <= cr.begin && cr.begin < off + incl;
-        const uint32_t m = __ballot_sync(kFullMask, hit);
-        if (m != 0) {
-            const int l = __ffs(m) - 1;
+        const uint32_t m0 = __ballot_sync(kFullMask, v > 0 && off + excl <= cr.begin && cr.begin < off + incl);
+        if (!found0 && m0 != 0) {
+            const int l = __ffs(m0) - 1;
             cr.b0 = base + l;
             cr.off0 = off + __shfl_sync(kFullMask, excl, l);
+            found0 = true;
+        }
+        const uint32_t ml = __ballot_sync(kFullMask, v > 0 && off + excl <= cr.end - 1 && cr.end - 1 < off + incl);
+        if (ml != 0) {
+            const int l = __ffs(ml) - 1;
+            cr.bl = base + l;
+            cr.offl = off + __shfl_sync(kFullMask, excl, l);
             return cr;
         }
         off += __shfl_sync(kFullMask, incl, 31);
@@ -161,13 +172,19 @@ struct Segment {
     long long uoff;  // line position of the unit's first tile
 };
 
-// Walks the segments of one CTA range in order.  Each role of the CTA runs its own walker;
-// all of them see the same sequence of segments.
+// Walks the segments of one CTA range: its last segment first (when the range has more than
+// one), then the others in line order.  The last segment usually starts a unit that the next
+// CTA finishes with its first segment, so both pieces of that unit are computed early and its
+// merge happens early too, not at the end of the kernel.  Each role of the CTA runs its own
+// walker; all of them see the same sequence of segments.
 struct SegmentWalker {
     const int32_t *lens;
     int B, UB, HB, L_max, T, window, Q;
     int b, n, nt;
     long long off, t, end;
+    bool last_first;  // the range's last segment is still to be returned first
+    int bl, nl, ntl, kl;
+    long long offl, tl, endl;
 
     __device__ void init(const DecodeParams &p, const CtaRange &cr) {
         lens = p.seq_lens;
@@ -182,9 +199,22 @@ struct SegmentWalker {
         end = cr.end;
         b = cr.b0;
         off = cr.off0;
+        last_first = false;
         if (t < end) {
             n = valid_len(lens[b], L_max, Q);
             nt = tiles_of(n - first_row(n, window), T);
+            bl = cr.bl;
+            offl = cr.offl;
+            nl = valid_len(lens[bl], L_max, Q);
+            ntl = tiles_of(nl - first_row(nl, window), T);
+            kl = static_cast<int>((end - 1 - offl) / ntl);
+            const long long uoffl = offl + static_cast<long long>(kl) * ntl;
+            if (uoffl > t) {  // more than one segment: the last one is [uoffl, end)
+                last_first = true;
+                tl = uoffl;
+                endl = end;
+                end = uoffl;
+            }
         } else {
             n = 0;
             nt = 0;
@@ -192,6 +222,22 @@ struct SegmentWalker {
     }
 
     __device__ bool next(Segment &s) {
+        if (last_first) {
+            last_first = false;
+            const int len = static_cast<int>(endl - tl);
+            s.b = bl;
+            s.kvh = kl / HB;
+            s.hb = kl - s.kvh * HB;
+            s.j0 = 0;
+            s.len = len;
+            s.n = nl;
+            s.first = first_row(nl, window);
+            s.unit = bl * UB + kl;
+            s.nt = ntl;
+            s.uoff = tl;
+            s.whole = len == ntl;
+            return true;
+        }
         if (t >= end) return false;
         while (t >= off + static_cast<long long>(nt) * UB) {
             off += static_cast<long long>(nt) * UB;
@@ -331,9 +377,11 @@ __device__ inline void merge_unit(const DecodeParams &p, const PendingPiece &u, 
 }
 
 // Bookkeeping of one group's partial pieces: record(...) right after the group barrier that
-// follows a partial piece's slot stores; finish(...) once, after the CTA's last segment.
+// follows a partial piece's slot stores; finish(...) after the CTA's second segment (the
+// walker returns the range's two partial pieces first) and once more after its last.
 struct PieceTickets {
     int n = 0;
+    int done = 0;
     int ticket[2] = {0, 0};
 
     __device__ void record(const DecodeParams &p, const Segment &sg, int group, int tid, PendingPiece *pend) {
@@ -347,7 +395,7 @@ struct PieceTickets {
     template <typename Bar>
     __device__ void finish(const DecodeParams &p, long long total, int group, int h0, int h1, int tid, int nthr,
                            PendingPiece *pend, int *flag, Bar bar) {
-        for (int k = 0; k < n && k < 2; ++k) {
+        for (int k = done; k < n && k < 2; ++k) {
             if (tid == 0) {
                 int c0, c1;
                 *flag = ticket[k] == unit_pieces(pend[k].uoff, pend[k].nt, total, p.G, c0, c1) - 1;
@@ -356,6 +404,7 @@ struct PieceTickets {
             if (*flag) merge_unit(p, pend[k], total, group, h0, h1, tid, nthr);
             bar();
         }
+        done = n;
     }
 };
 
