@@ -15,11 +15,12 @@
 // rounding residual) side by side, summed when the tile is read back, so it carries ~16
 // significant bits rather than 8.  NH is the group's head count rounded up to a power of two
 // (1..64) and RP = max(16, NH) the UMMA N; padded heads are computed and ignored.
-// Roles (64 + 128 * NWG threads):
+// Roles (64 + 128 * NWG + 32 threads):
 //   warp 0       TMA producer (q of each unit, K/V tiles); also owns the tensor memory
 //   warp 1       UMMA issuer (one elected thread, event loop)
 //   warps 2..    NWG softmax / accumulation / epilogue warpgroups of 128 threads, each owning
 //                a slice of the group's query heads (one warpgroup up to 16 heads)
+//   last warp    ticket warp: takes the tickets of the pieces cut from units (schedule.cuh)
 // Every wait is bounded; on a timeout the CTA drains its in-flight copies and UMMAs, frees
 // its tensor memory, sets GQA_STATUS_WAIT_TIMEOUT and returns.
 #include <cstdint>
@@ -59,7 +60,8 @@ struct TcCfg {
     // independent, so the groups split them and never exchange data).
     static constexpr int NWG = NH >= 32 ? NH / 16 : 1;
     static constexpr int NHW = NH / NWG;              // heads per warpgroup
-    static constexpr int THREADS = 64 + 128 * NWG;
+    static constexpr int TICKET_WARP = 2 + 4 * NWG;
+    static constexpr int THREADS = 64 + 128 * NWG + 32;
     static constexpr int NHW4 = (NHW + 3) / 4;
     static constexpr int LOG2NHW = NHW >= 16 ? 4 : NHW >= 8 ? 3 : NHW >= 4 ? 2 : NHW >= 2 ? 1 : 0;
 
@@ -68,12 +70,13 @@ struct TcCfg {
         uint64_t q_full[2], q_empty[2];
         uint64_t s_full[2], s_empty[2], p_full[2], o_full[2], o_empty[2];
         uint64_t mma_done;
+        uint64_t pc_full[kPieceGroups][2];  // a group's partial piece is in its slot
+        uint64_t tk_done[kPieceGroups][2];  // its ticket is taken: tk_last says if it was the last
+        int tk_last[kPieceGroups][2];  // a group's partial piece is in its slot
         uint32_t tmem_base;
         int abort;
         int b0, bl;
         long long begin, end, off0, offl, total;
-        int pflag[kPieceGroups];
-        PendingPiece pend[kPieceGroups][2];
         float4 wmax[NWG][2][4][NHW4];  // per group, tile parity, warp: per-head warp maxima
         float lsum[NWG][4][NHW];
     };
@@ -164,6 +167,12 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mbar_init(&sm->o_empty[j], 4 * C::NWG);
         }
         mbar_init(&sm->mma_done, 1);
+        for (int g = 0; g < kPieceGroups; ++g) {
+            mbar_init(&sm->pc_full[g][0], 1);
+            mbar_init(&sm->pc_full[g][1], 1);
+            mbar_init(&sm->tk_done[g][0], 1);
+            mbar_init(&sm->tk_done[g][1], 1);
+        }
         sm->abort = 0;
         fence_mbarrier_init();
     }
@@ -419,6 +428,9 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             umma_commit(&sm->mma_done);
             wait_bounded(&sm->mma_done, 0, nullptr, kDrainNs);
         }
+    } else if (warp == C::TICKET_WARP) {
+        // ------------------------------------------------------------------ ticket warp
+        run_ticket_warp<C::NWG>(p, cr, sm->pc_full, sm->tk_done, sm->tk_last, lane, abort_flag, budget);
     } else {
         // ------------------------------------------------------------------ softmax warps
         // NWG warpgroups of four warps; warpgroup g owns query heads [g*NHW, (g+1)*NHW) of the
@@ -441,8 +453,13 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         int i = 0;
         bool ok = true;
         float O[NHW], l[NHW], m_run[NHW], alpha[NHW];
-        PieceTickets tickets;
-        int nseg = 0;
+        int npart = 0, nmerged = 0;  // partial pieces handed to the ticket warp, reports taken
+        PendingPiece parts[2];
+        auto merge_in = [&](bool block) {
+            return merge_reported(p, cr.total, wg, hbase, hbase + NHW, sm_tid - 128 * wg, 128, sm->tk_done[wg], sm->tk_last[wg],
+                                  parts, npart, nmerged, block, abort_flag, budget,
+                                  [&](bool pred) { return named_bar_any(bar_id, 128, pred); });
+        };
         // units with no rows get zeros (while the first tiles are still on their way)
         zero_empty_units(p, blockIdx.x, sm_tid, 128 * C::NWG);
         while (ok && w.next(sg)) {
@@ -666,22 +683,19 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     }
                 }
             }
-            // the next piece rewrites lsum only after every thread has read it (and the slot
-            // stores are ordered before the ticket)
+            // the next piece rewrites lsum only after every thread has read it, and the slot
+            // is complete before the ticket warp is told
             named_bar_sync(bar_id, 128);
-            if (!sg.whole) tickets.record(p, sg, wg, sm_tid - 128 * wg, sm->pend[wg]);
-            // the range's partial pieces come first: merge what they complete right away
-            if (++nseg == 2)
-                tickets.finish(p, cr.total, wg, hbase, hbase + NHW, sm_tid - 128 * wg, 128, sm->pend[wg],
-                               &sm->pflag[wg], [&] { named_bar_sync(bar_id, 128); });
+            if (!sg.whole) {
+                if (sm_tid == 128 * wg && npart < 2) mbar_arrive(&sm->pc_full[wg][npart]);
+                if (npart < 2) parts[npart] = PendingPiece{sg.uoff, sg.unit, sg.b, sg.kvh, sg.hb, sg.nt};
+                ++npart;
+            }
+            // merge what an earlier piece completed, if its ticket is back
+            merge_in(false);
         }
-        if (!ok) {
-            fail();
-        } else {
-            // units cut into pieces are merged by the CTA holding the last ticket
-            tickets.finish(p, cr.total, wg, hbase, hbase + NHW, sm_tid - 128 * wg, 128, sm->pend[wg],
-                           &sm->pflag[wg], [&] { named_bar_sync(bar_id, 128); });
-        }
+        if (ok && !merge_in(true)) ok = false;
+        if (!ok) fail();
     }
 
     tc_fence_before_sync();

@@ -72,7 +72,8 @@ struct Tc8Cfg {
     // a tile's softmax takes the time of 128 rows
     static constexpr int RS = RT;
     static constexpr int NSW = NWG * RS;               // softmax warpgroups
-    static constexpr int THREADS = 64 + 128 * NSW;
+    static constexpr int TICKET_WARP = 2 + 4 * NSW;    // the ticket warp (schedule.cuh)
+    static constexpr int THREADS = 64 + 128 * NSW + 32;
     static constexpr int NHW4 = (NHW + 3) / 4;
     static constexpr int LOG2NHW = NHW >= 16 ? 4 : NHW >= 8 ? 3 : NHW >= 4 ? 2 : NHW >= 2 ? 1 : 0;
 
@@ -81,12 +82,13 @@ struct Tc8Cfg {
         uint64_t q_full[2], q_empty[2], qf_empty[2];
         uint64_t s_full[2], s_empty[2], p_full[2], o_full[2], o_empty[2];
         uint64_t mma_done;
+        uint64_t pc_full[kPieceGroups][2];  // a group's partial piece is in its slot
+        uint64_t tk_done[kPieceGroups][2];  // its ticket is taken: tk_last says if it was the last
+        int tk_last[kPieceGroups][2];  // a head slice's partial piece is in its slot
         uint32_t tmem_base;
         int abort;
         int b0, bl;
         long long begin, end, off0, offl, total;
-        int pflag[kPieceGroups];
-        PendingPiece pend[kPieceGroups][2];
         float qf[2][RP];                    // score factor of each column: scale * k_scale / c_h
         float vsc[2];                       // v_scale of the unit's key/value head
         float4 wmax[NWG][2][4 * RS][NHW4];  // per head slice, S buffer, warp: warp maxima
@@ -206,6 +208,12 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             mbar_init(&sm->o_empty[j], 4 * C::NWG);     // the first row half folds O
         }
         mbar_init(&sm->mma_done, 1);
+        for (int g = 0; g < kPieceGroups; ++g) {
+            mbar_init(&sm->pc_full[g][0], 1);
+            mbar_init(&sm->pc_full[g][1], 1);
+            mbar_init(&sm->tk_done[g][0], 1);
+            mbar_init(&sm->tk_done[g][1], 1);
+        }
         sm->abort = 0;
         fence_mbarrier_init();
     }
@@ -514,6 +522,9 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             umma_commit(&sm->mma_done);
             wait_bounded(&sm->mma_done, 0, nullptr, kDrainNs8);
         }
+    } else if (warp == C::TICKET_WARP) {
+        // ------------------------------------------------------------------ ticket warp
+        run_ticket_warp<C::NWG>(p, cr, sm->pc_full, sm->tk_done, sm->tk_last, lane, abort_flag, budget);
     } else {
         // ------------------------------------------------------------------ softmax warps
         // Every softmax thread owns one row of each tile.  NWG warpgroups split the heads
@@ -544,8 +555,13 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         int i = 0, sidx = 0;
         bool ok = true;
         float O[NHW], l[NHW], m_run[NHW], alpha[NHW], f[NHW];
-        PieceTickets tickets;
-        int nseg = 0;
+        int npart = 0, nmerged = 0;  // partial pieces handed to the ticket warp, reports taken
+        PendingPiece parts[2];
+        auto merge_in = [&](bool block) {
+            return merge_reported(p, cr.total, wg, hbase, hbase + NHW, sm_tid, NBAR, sm->tk_done[wg], sm->tk_last[wg],
+                                  parts, npart, nmerged, block, abort_flag, budget,
+                                  [&](bool pred) { return named_bar_any(bar_id, NBAR, pred); });
+        };
         // units with no rows get zeros (while the first tiles are still on their way)
         zero_empty_units(p, blockIdx.x, threadIdx.x - 64, 128 * C::NSW);
         // O of tile t folded into the running sum, scaled by `scale_by` (first row half only)
@@ -765,22 +781,19 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                     }
                 }
             }
-            // the next unit rewrites lsum only after every thread has read it (and the slot
-            // stores are ordered before the ticket)
+            // the next unit rewrites lsum only after every thread has read it, and the slot is
+            // complete before the ticket warp is told
             named_bar_sync(bar_id, NBAR);
-            if (!sg.whole) tickets.record(p, sg, wg, sm_tid, sm->pend[wg]);
-            // the range's partial pieces come first: merge what they complete right away
-            if (++nseg == 2)
-                tickets.finish(p, cr.total, wg, hbase, hbase + NHW, sm_tid, NBAR, sm->pend[wg], &sm->pflag[wg],
-                               [&] { named_bar_sync(bar_id, NBAR); });
+            if (!sg.whole) {
+                if (sm_tid == 0 && npart < 2) mbar_arrive(&sm->pc_full[wg][npart]);
+                if (npart < 2) parts[npart] = PendingPiece{sg.uoff, sg.unit, sg.b, sg.kvh, sg.hb, sg.nt};
+                ++npart;
+            }
+            // merge what an earlier piece completed, if its ticket is back
+            merge_in(false);
         }
-        if (!ok) {
-            fail();
-        } else {
-            // units cut into pieces are merged by the CTA holding the last ticket
-            tickets.finish(p, cr.total, wg, hbase, hbase + NHW, sm_tid, NBAR, sm->pend[wg], &sm->pflag[wg],
-                           [&] { named_bar_sync(bar_id, NBAR); });
-        }
+        if (ok && !merge_in(true)) ok = false;
+        if (!ok) fail();
     }
 
     tc_fence_before_sync();

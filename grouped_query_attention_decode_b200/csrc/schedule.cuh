@@ -408,6 +408,54 @@ struct PieceTickets {
     }
 };
 
+// The ticket warp of a CTA.  Each group of softmax threads (NG of them, one per head slice)
+// stores a partial piece's slot and arrives on pc_full[group][k] (k: the piece's place among
+// the CTA's partial pieces, at most two); this warp then takes the group's ticket for the unit
+// -- the atomic's release covers the slot stores the barrier made it observe, its acquire the
+// other pieces' -- and reports whether it was the last one in tk_last[group][k], arriving on
+// tk_done[group][k].  The softmax threads never wait on the atomic; they merge the units
+// reported to them (merge_reported) with all their threads.
+template <int NG>
+__device__ void run_ticket_warp(const DecodeParams &p, const CtaRange &cr, uint64_t (*pc_full)[2],
+                                uint64_t (*tk_done)[2], int (*tk_last)[2], int lane,
+                                const volatile int *abort_flag, uint64_t budget) {
+    SegmentWalker w;
+    w.init(p, cr);
+    Segment sg;
+    int k = 0;
+    while (k < 2 && w.next(sg)) {
+        if (sg.whole) continue;
+        for (int g = 0; g < NG; ++g) {
+            const bool got = wait_bounded(&pc_full[g][k], 0, abort_flag, budget);
+            if (!__all_sync(kFullMask, got)) return;  // the softmax side failed; it reports it
+            if (lane == 0) {
+                int c0, c1;
+                tk_last[g][k] = take_ticket(p, sg.unit, g) == unit_pieces(sg.uoff, sg.nt, cr.total, p.G, c0, c1) - 1;
+                mbar_arrive(&tk_done[g][k]);
+            }
+        }
+        ++k;
+    }
+}
+
+// Softmax side of the ticket warp, for one group of nthr threads: the units whose last ticket
+// was reported for the group's partial pieces [done, n) are merged, in order.  Non-blocking
+// (block = false) it stops at the first piece whose report is not in yet; blocking it waits
+// for each.  bar_any(pred) is a barrier of the group that returns whether pred held in any
+// thread, so every decision is the group's.  Returns false when a blocking wait gave up.
+template <typename BarAny>
+__device__ bool merge_reported(const DecodeParams &p, long long total, int group, int h0, int h1, int tid,
+                               int nthr, uint64_t *tk_done, const int *tk_last, const PendingPiece *pp,
+                               int n, int &done, bool block, const volatile int *abort_flag,
+                               uint64_t budget, BarAny bar_any) {
+    for (; done < n && done < 2; ++done) {
+        const bool got = block ? wait_bounded(&tk_done[done], 0, abort_flag, budget) : mbar_test_wait(&tk_done[done], 0);
+        if (bar_any(!got)) return !block;
+        if (tk_last[done]) merge_unit(p, pp[done], total, group, h0, h1, tid, nthr);
+    }
+    return true;
+}
+
 // Units with no rows (a sequence of length 0, or one refused as out of range) get zero
 // output; CTA `cta` of G covers units cta, cta + G, ...
 __device__ inline void zero_empty_units(const DecodeParams &p, int cta, int tid, int nthr) {
