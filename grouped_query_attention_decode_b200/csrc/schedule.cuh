@@ -329,49 +329,85 @@ __device__ inline void merge_unit(const DecodeParams &p, const PendingPiece &u, 
     const float *base = p.ws + p.hdr_floats + static_cast<long long>(u.unit) * p.slot_floats;
     const bool some_empty = total < p.G;
     const int nvec = (h1 - h0) * d / 4;
-    // four vectors per thread per round, all loaded before any store
-    for (int v0 = tid; v0 < nvec; v0 += 4 * nthr) {
-        float4 res[4];
-        long long dst[4];
+    // The non-empty pieces c0 .. c1 in line order (a CTA with an empty range holds none).
+    auto next_piece = [&](int c) {
+        while (c <= c1 && some_empty && cta_range_begin(c, total, p.G) >= cta_range_begin(c + 1, total, p.G)) ++c;
+        return c;
+    };
+    // kVR vectors per thread per round.  Each piece's values for all of them are loaded at
+    // once, one piece ahead of the arithmetic, so a round costs about one L2 round trip rather
+    // than one per vector and piece; the arithmetic per vector is the one-pass merge in line
+    // order.
+    constexpr int kVR = 2;
+    for (int v0 = tid; v0 < nvec; v0 += kVR * nthr) {
+        int idx[kVR], hh[kVR];
+        long long dst[kVR];
+        float M[kVR], den[kVR];
+        float4 num[kVR];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < kVR; ++j) {
             const int v = v0 + j * nthr;
             dst[j] = -1;
-            res[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+            idx[j] = 0;
+            hh[j] = 0;
+            M[j] = -INFINITY;
+            den[j] = 0.f;
+            num[j] = make_float4(0.f, 0.f, 0.f, 0.f);
             if (v >= nvec) continue;
-            const int idx = h0 * d + 4 * v;
-            const int h = idx / d;
-            const long long orow = out_row(p, u.b, u.kvh, u.hb, h);
-            if (orow < 0) continue;
-            float M = -INFINITY, den = 0.f;
-            float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int c = c0; c <= c1; ++c) {
-                if (some_empty && cta_range_begin(c, total, p.G) >= cta_range_begin(c + 1, total, p.G)) continue;
-                const float *sl = base + static_cast<long long>(c) * p.slot_floats;
-                const float m = __ldcg(sl + nh * d + h);
-                const float l = __ldcg(sl + nh * d + nh + h);
-                const float4 o = __ldcg(reinterpret_cast<const float4 *>(sl + idx));
-                if (m == -INFINITY) continue;
-                if (m > M) {
-                    const float sc = M == -INFINITY ? 0.f : ex2_approx(M - m);
-                    num.x *= sc; num.y *= sc; num.z *= sc; num.w *= sc;
-                    den *= sc;
-                    M = m;
+            idx[j] = h0 * d + 4 * v;
+            hh[j] = idx[j] / d;
+            const long long orow = out_row(p, u.b, u.kvh, u.hb, hh[j]);
+            if (orow >= 0) dst[j] = orow * d + (idx[j] - hh[j] * d);
+        }
+        float m_n[kVR], l_n[kVR];
+        float4 o_n[kVR];
+        auto load = [&](int c) {
+            const float *sl = base + static_cast<long long>(c) * p.slot_floats;
+#pragma unroll
+            for (int j = 0; j < kVR; ++j)
+                if (dst[j] >= 0) {
+                    m_n[j] = __ldcg(sl + nh * d + hh[j]);
+                    l_n[j] = __ldcg(sl + nh * d + nh + hh[j]);
+                    o_n[j] = __ldcg(reinterpret_cast<const float4 *>(sl + idx[j]));
                 }
-                const float wgt = ex2_approx(m - M);
-                num.x = fmaf(wgt, o.x, num.x);
-                num.y = fmaf(wgt, o.y, num.y);
-                num.z = fmaf(wgt, o.z, num.z);
-                num.w = fmaf(wgt, o.w, num.w);
-                den = fmaf(wgt, l, den);
+        };
+        int c = next_piece(c0);
+        if (c <= c1) load(c);
+        while (c <= c1) {
+            float m_c[kVR], l_c[kVR];
+            float4 o_c[kVR];
+#pragma unroll
+            for (int j = 0; j < kVR; ++j) {
+                m_c[j] = m_n[j];
+                l_c[j] = l_n[j];
+                o_c[j] = o_n[j];
             }
-            const float inv = 1.f / den;
-            res[j] = make_float4(num.x * inv, num.y * inv, num.z * inv, num.w * inv);
-            dst[j] = orow * d + (idx - h * d);
+            c = next_piece(c + 1);
+            if (c <= c1) load(c);
+#pragma unroll
+            for (int j = 0; j < kVR; ++j) {
+                if (dst[j] < 0 || m_c[j] == -INFINITY) continue;
+                if (m_c[j] > M[j]) {
+                    const float sc = M[j] == -INFINITY ? 0.f : ex2_approx(M[j] - m_c[j]);
+                    num[j].x *= sc; num[j].y *= sc; num[j].z *= sc; num[j].w *= sc;
+                    den[j] *= sc;
+                    M[j] = m_c[j];
+                }
+                const float wgt = ex2_approx(m_c[j] - M[j]);
+                num[j].x = fmaf(wgt, o_c[j].x, num[j].x);
+                num[j].y = fmaf(wgt, o_c[j].y, num[j].y);
+                num[j].z = fmaf(wgt, o_c[j].z, num[j].z);
+                num[j].w = fmaf(wgt, o_c[j].w, num[j].w);
+                den[j] = fmaf(wgt, l_c[j], den[j]);
+            }
         }
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-            if (dst[j] >= 0) *reinterpret_cast<float4 *>(p.out + dst[j]) = res[j];
+        for (int j = 0; j < kVR; ++j)
+            if (dst[j] >= 0) {
+                const float inv = 1.f / den[j];
+                *reinterpret_cast<float4 *>(p.out + dst[j]) =
+                    make_float4(num[j].x * inv, num[j].y * inv, num[j].z * inv, num[j].w * inv);
+            }
     }
     if (tid == 0) p.cnt[static_cast<long long>(u.unit) * kPieceGroups + group] = 0;
 }
