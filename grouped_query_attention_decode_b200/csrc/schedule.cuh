@@ -1,4 +1,4 @@
-// Work partition shared by the split-KV kernels and the combine kernel.
+// Work partition and piece merge shared by the split-KV kernels.
 //
 // The decode work is cut into tiles of T cached rows.  A "unit" is one (sequence b, key/value
 // head j, block of up to 64 query heads of j's group); a unit has ceil(n_b / T) tiles.  Units
@@ -8,9 +8,9 @@
 // so every CTA streams the same number of tiles (to within one) whatever the length mix.  A
 // CTA range may cut a unit; each (CTA, unit) piece produces a partial result in workspace
 // slot (CTA index + unit index), which is unique because both indices grow along the line.
-// A unit covered by a single piece is finished by that CTA; the others are merged by the
-// combine kernel.  Every kernel derives the same partition from seq_lens on the device, so
-// the host never needs the lengths.
+// A unit covered by a single piece is finished by that CTA; a unit cut into pieces is merged
+// inside the same kernel (piece merge, below).  Every kernel derives the same partition from
+// seq_lens on the device, so the host never needs the lengths.
 #pragma once
 
 #include <cstdint>
@@ -318,8 +318,8 @@ __device__ __forceinline__ int take_ticket(const DecodeParams &p, int unit, int 
 }
 
 // The group (threads tid < nthr) that took a unit's last ticket merges that unit's columns
-// [h0, h1): a one-pass log-sum-exp over the pieces' slots, four outputs per step, and puts the
-// counter back to zero.
+// [h0, h1): a one-pass log-sum-exp over the pieces' slots, four outputs (one float4) per
+// vector, and puts the counter back to zero.
 __device__ inline void merge_unit(const DecodeParams &p, const PendingPiece &u, long long total,
                                   int group, int h0, int h1, int tid, int nthr) {
     int c0, c1;
