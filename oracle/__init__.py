@@ -22,6 +22,7 @@ _LIB = os.path.join(_HERE, "liboracle.so")
 
 APPEND_OVERFLOW = 1
 SEQLEN_RANGE = 2
+PAGE_RANGE = 4  # a block-table entry outside the pool for a row below the length
 
 
 def build(src: str = _SRC, out: str = _LIB) -> str:
@@ -215,11 +216,16 @@ class Oracle:
                                         H_kv, d, self._ip(status))
         return int(status[0])
 
-    def decode_paged(self, q, k_pool, v_pool, block_table, seq_lens, scale: float):
-        """The paged decode: gather each sequence's rows from the pool, then decode."""
+    def decode_paged(self, q, k_pool, v_pool, block_table, seq_lens, scale: float,
+                     return_status: bool = False):
+        """The paged decode: gather each sequence's rows from the pool, then decode.  With
+        return_status, also returns the status bits of the gathers and the decode (PAGE_RANGE
+        when a block-table entry for a row below the length lies outside the pool; that row is
+        then gathered as zeros)."""
         kc, st1 = self.paged_gather(k_pool, block_table, seq_lens)
         vc, st2 = self.paged_gather(v_pool, block_table, seq_lens)
-        return self.decode(q, kc, vc, seq_lens, scale)
+        out, st3 = self.decode(q, kc, vc, seq_lens, scale, return_status=True)
+        return (out, st1 | st2 | st3) if return_status else out
 
     # ------------------------------------------------------------------ FP8 (e4m3) cache
     @staticmethod
@@ -304,10 +310,11 @@ class Oracle:
         return self.decode_window(q, kc, vc, seq_lens, window, scale, nthreads=nthreads)
 
     def decode_paged_fp8(self, q, k_pool, v_pool, k_scale, v_scale, block_table, seq_lens,
-                         scale: float):
+                         scale: float, return_status: bool = False):
         """Paged decode over e4m3 pools: dequantise the pools, gather, decode."""
         return self.decode_paged(q, self.dequantize(k_pool, k_scale),
-                                 self.dequantize(v_pool, v_scale), block_table, seq_lens, scale)
+                                 self.dequantize(v_pool, v_scale), block_table, seq_lens, scale,
+                                 return_status=return_status)
 
 
 _default: Oracle | None = None

@@ -348,6 +348,21 @@ def pin_paged(o):
     full = l2.copy()
     full[2] = L  # a full sequence is refused too
     assert o.kv_append_paged(kn, vn, kpool2, vpool2, table2, full) & 1 and full[2] == L
+    # the decode reports a block-table entry outside the pool for a row it must read, and
+    # gathers that row as zeros; an entry past the length is never looked at
+    out_ok, st_ok = o.decode_paged(q, kpool2, vpool2, table2, lens, 0.25, return_status=True)
+    assert st_ok == 0 and np.array_equal(out_ok, base)
+    bad2 = table2.copy()
+    bad2[0, 1] = -1  # rows 8..15 of sequence 0 (length 39)
+    out_bad, st_bad = o.decode_paged(q, kpool2, vpool2, bad2, lens, 0.25, return_status=True)
+    assert st_bad & 4
+    Kz, Vz = Kc.copy(), Vc.copy()
+    Kz[0, P:2 * P] = 0.0
+    Vz[0, P:2 * P] = 0.0
+    assert np.array_equal(out_bad, o.decode(q, Kz, Vz, lens, 0.25))
+    unused = table2.copy()
+    unused[1, max_pages - 1] = n_pages + 7  # sequence 1 has one row: its last page is unused
+    assert o.decode_paged(q, kpool2, vpool2, unused, lens, 0.25, return_status=True)[1] == 0
 
 
 def pin_multi_query(o):

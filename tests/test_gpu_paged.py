@@ -9,6 +9,7 @@ import pytest
 import torch
 
 import grouped_query_attention_decode_b200 as gqa
+import oracle as oracle_mod
 from gpu_helpers import TOL
 from grouped_query_attention_decode_b200 import inputs
 
@@ -71,17 +72,23 @@ def test_paged_full_size_llama(oracle):
     _step(oracle, w, None, w.page_size, bs=[0, 7, 15])
 
 
-def test_paged_bad_page_is_reported():
+def test_paged_bad_page_is_reported(oracle):
     w = inputs.custom("pagedbad", B=2, H_q=16, H_kv=4, d=128, L_max=256, dtype=torch.bfloat16, seed=54)
     x = inputs.make_inputs(w, lengths=[256, 40])
     pg = inputs.make_paged(x, 32)
     bt = pg["block_table"].clone()
     bt[1, 0] = 10_000  # no such page
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    gqa.decode_paged(x["q"].cuda(), pg["k_pool"].cuda(), pg["v_pool"].cuda(), bt.cuda(),
-                     x["lengths"].cuda(), x["scale"], status=status)
+    out = gqa.decode_paged(x["q"].cuda(), pg["k_pool"].cuda(), pg["v_pool"].cuda(), bt.cuda(),
+                           x["lengths"].cuda(), x["scale"], status=status)
     torch.cuda.synchronize()
     assert int(status.item()) & gqa.STATUS_PAGE_RANGE
+    # the oracle reports the same entry; the sequence with a valid table still matches it
+    ref, st = oracle.decode_paged(x["q"].double().numpy(), pg["k_pool"].double().numpy(),
+                                  pg["v_pool"].double().numpy(), bt.numpy(), x["lengths"].numpy(),
+                                  x["scale"], return_status=True)
+    assert st & oracle_mod.PAGE_RANGE
+    assert float(np.max(np.abs(out[0].cpu().double().numpy() - ref[0]))) <= TOL[w.dtype]
 
 
 def test_paged_rejects_unsupported_page_size():
