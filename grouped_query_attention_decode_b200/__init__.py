@@ -33,7 +33,7 @@ EXPORTED = ("gqa_kv_append", "gqa_decode_workspace_size", "gqa_decode", "gqa_sta
             "gqa_decode_window", "gqa_kv_append_paged", "gqa_decode_paged",
             "gqa_kv_append_multi", "gqa_decode_multi_workspace_size", "gqa_decode_multi",
             "gqa_kv_append_fp8", "gqa_kv_append_paged_fp8", "gqa_decode_fp8",
-            "gqa_decode_paged_fp8")
+            "gqa_decode_paged_fp8", "gqa_kv_append_decode")
 
 
 class GQAError(RuntimeError):
@@ -65,6 +65,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gqa_decode.argtypes = [vp, vp, vp, i32p, c_int, c_int, c_int, c_int, c_int,
                                ctypes.c_float, c_int, vp, vp, c_size, i32p, vp]
     lib.gqa_decode.restype = c_int
+    lib.gqa_kv_append_decode.argtypes = [vp, vp, vp, vp, vp, i32p, i32p, c_int, c_int, c_int,
+                                         c_int, c_int, ctypes.c_float, c_int, vp, vp, c_size,
+                                         i32p, vp]
+    lib.gqa_kv_append_decode.restype = c_int
     lib.gqa_decode_window.argtypes = [vp, vp, vp, i32p, c_int, c_int, c_int, c_int, c_int, c_int,
                                       ctypes.c_float, c_int, vp, vp, c_size, i32p, vp]
     lib.gqa_decode_window.restype = c_int
@@ -170,6 +174,24 @@ def decode(q, k_cache, v_cache, seq_lens, scale: float, out=None, workspace=None
         _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens), B, H_q, H_kv, d, L_max,
         float(scale), _dtype(k_cache), _ptr(out), _ptr(workspace), workspace.numel(),
         _ptr(status), _stream(stream)))
+    return out
+
+
+def kv_append_decode(q, k_new, v_new, k_cache, v_cache, seq_lens, seq_lens_out, scale: float,
+                     out=None, workspace=None, status=None, stream=None) -> torch.Tensor:
+    """gqa_kv_append_decode: append k_new/v_new at row seq_lens[b] and attend the rows up to and
+    including it, in one launch; the new lengths go to ``seq_lens_out`` (``seq_lens`` is only
+    read).  Returns ``out`` [B, H_q, d] float32."""
+    B, H_q, d = q.shape
+    _, L_max, H_kv, _ = k_cache.shape
+    if out is None:
+        out = torch.empty((B, H_q, d), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(B, H_q, H_kv, d, k_cache.dtype, device=q.device)
+    _check(load_library().gqa_kv_append_decode(
+        _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens),
+        _ptr(seq_lens_out), B, H_q, H_kv, d, L_max, float(scale), _dtype(k_cache), _ptr(out),
+        _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream)))
     return out
 
 

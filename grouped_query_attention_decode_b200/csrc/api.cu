@@ -50,7 +50,7 @@ int current_sm_count(int *dev_out) {
 
 struct Geometry {
     int r, rb, RB, HB, UB;
-    long long units, slots, slot_floats, hdr_floats, cnt_floats;
+    long long units, slots, slot_floats, slot_base;
     size_t bytes;
 };
 
@@ -68,10 +68,10 @@ Geometry geometry(int B, int H_q, int H_kv, int d, int G, int Q = 1) {
     // O [RB][d], m [RB], l [RB], rounded up to whole 16-byte vectors (the merge reads o with
     // 16-byte loads)
     g.slot_floats = (static_cast<long long>(g.RB) * (d + 2) + 3) / 4 * 4;
-    // int64 header [B + 1], then the per-unit piece counters, each region a 256-byte multiple
-    g.cnt_floats = ((static_cast<long long>(B) + 1) * 8 + 255) / 256 * 64;
-    g.hdr_floats = g.cnt_floats + (g.units * kPieceGroups * 4 + 255) / 256 * 64;
-    g.bytes = static_cast<size_t>((g.hdr_floats + g.slots * g.slot_floats) * 4 + 255) / 256 * 256;
+    // the per-unit piece counters (int32, kPieceGroups per unit) at offset 0, then the slots
+    // from the next 256-byte boundary
+    g.slot_base = (g.units * kPieceGroups * 4 + 255) / 256 * 64;
+    g.bytes = static_cast<size_t>((g.slot_base + g.slots * g.slot_floats) * 4 + 255) / 256 * 256;
     return g;
 }
 
@@ -219,8 +219,8 @@ size_t gqa::decode_counter_region(int B, int H_q, int H_kv, int d, size_t *offse
     const int sms = current_sm_count(&dev);
     if (sms <= 0) return 0;
     const Geometry g = geometry(B, H_q, H_kv, d, sms);
-    *offset = static_cast<size_t>(g.cnt_floats) * 4;
-    return static_cast<size_t>(g.hdr_floats - g.cnt_floats) * 4;
+    *offset = 0;
+    return static_cast<size_t>(g.slot_base) * 4;
 }
 
 extern "C" size_t gqa_decode_workspace_size(int B, int H_q, int H_kv, int d, gqa_dtype_t dtype) {
@@ -239,11 +239,19 @@ struct PagedArgs {
     int max_pages = 0, page_size = 0, n_pages = 0;
 };
 
+// The append fused into the decode (k_new == nullptr: none).
+struct AppendArgs {
+    const void *k_new = nullptr, *v_new = nullptr;
+    void *k_cache = nullptr, *v_cache = nullptr;
+    int32_t *lens_out = nullptr;
+};
+
 int decode_impl(const void *q, const void *k_cache, const void *v_cache, const int32_t *seq_lens,
                 int B, int H_q, int H_kv, int d, int L_max, int window, float scale,
                 gqa_dtype_t dtype, float *out, void *workspace, size_t workspace_bytes,
                 int32_t *status, cudaStream_t stream, const PagedArgs &pg = PagedArgs(),
-                int Q = 1, const float *k_scale = nullptr, const float *v_scale = nullptr) {
+                int Q = 1, const float *k_scale = nullptr, const float *v_scale = nullptr,
+                bool dry_run = false, const AppendArgs &ap = AppendArgs()) {
     if (!q || !k_cache || !v_cache || !seq_lens || !out) return GQA_ERR_NULL;
     const bool fp8 = k_scale != nullptr;
     const int rc = check_shape(B, H_q, H_kv, d, L_max, dtype, fp8);
@@ -261,7 +269,7 @@ int decode_impl(const void *q, const void *k_cache, const void *v_cache, const i
     if (Q < 1 || Q > 64) return GQA_ERR_SHAPE;
     const Geometry g = geometry(B, H_q, H_kv, d, sms, Q);
     if (workspace_bytes < g.bytes) return GQA_ERR_WORKSPACE;
-    if (g.slot_floats % 4 != 0 || g.hdr_floats % 4 != 0) return GQA_ERR_SHAPE;  // 16-byte slot vectors
+    if (g.slot_floats % 4 != 0 || g.slot_base % 4 != 0) return GQA_ERR_SHAPE;  // 16-byte slot vectors
 
     DecodeParams p;
     p.seq_lens = seq_lens;
@@ -283,6 +291,12 @@ int decode_impl(const void *q, const void *k_cache, const void *v_cache, const i
     p.T = fp8 ? tc8_tile_rows(g.RB) : (dtype == GQA_DTYPE_BF16 ? 128 : 64);
     p.k_scale = k_scale;
     p.v_scale = v_scale;
+    p.k_new = ap.k_new;
+    p.v_new = ap.v_new;
+    p.k_cache = ap.k_cache;
+    p.v_cache = ap.v_cache;
+    p.lens_out = ap.lens_out;
+    p.append = ap.k_new != nullptr ? 1 : 0;
     p.window = window;
     p.block_table = pg.block_table;
     p.max_pages = pg.max_pages;
@@ -296,8 +310,8 @@ int decode_impl(const void *q, const void *k_cache, const void *v_cache, const i
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     p.wait_ns = g_wait_ns.load();
     p.slot_floats = g.slot_floats;
-    p.hdr_floats = g.hdr_floats;
-    p.cnt = reinterpret_cast<int32_t *>(static_cast<float *>(workspace) + g.cnt_floats);
+    p.slot_base = g.slot_base;
+    p.cnt = static_cast<int32_t *>(workspace);
 
     cudaEvent_t ev0 = g_ev_before.load(), ev1 = g_ev_after.load();
     const bool profile = ev0 != nullptr && ev1 != nullptr;
@@ -313,6 +327,7 @@ int decode_impl(const void *q, const void *k_cache, const void *v_cache, const i
             !encode_cache_map8(&maps.v, v_cache, outer_dim, H_kv, d, rows_dim, box) ||
             !encode_cache_map8(&maps.v8, v_cache, outer_dim, H_kv, d, rows_dim, 8))
             return GQA_ERR_SHAPE;
+        if (dry_run) return GQA_OK;
         if (profile && cudaEventRecord(ev0, stream) != cudaSuccess) return GQA_ERR_CUDA;
         res = launch_split_tc8(maps, q, p, stream);
     } else if (dtype == GQA_DTYPE_BF16) {
@@ -330,9 +345,11 @@ int decode_impl(const void *q, const void *k_cache, const void *v_cache, const i
             !encode_cache_map(&maps.v, v_cache, outer_dim, H_kv, d, rows_dim, box) ||
             !encode_cache_map(&maps.v8, v_cache, outer_dim, H_kv, d, rows_dim, 8))
             return GQA_ERR_SHAPE;
+        if (dry_run) return GQA_OK;
         if (profile && cudaEventRecord(ev0, stream) != cudaSuccess) return GQA_ERR_CUDA;
         res = launch_split_tc(maps, p, stream);
     } else {
+        if (dry_run) return GQA_OK;
         if (profile && cudaEventRecord(ev0, stream) != cudaSuccess) return GQA_ERR_CUDA;
         res = launch_split_f32(p, static_cast<const float *>(q), static_cast<const float *>(k_cache),
                                static_cast<const float *>(v_cache), stream);
@@ -344,12 +361,48 @@ int decode_impl(const void *q, const void *k_cache, const void *v_cache, const i
 
 }  // namespace
 
+int gqa::decode_check(const void *q, const void *k_cache, const void *v_cache,
+                      const int32_t *seq_lens, int B, int H_q, int H_kv, int d, int L_max,
+                      float scale, gqa_dtype_t dtype, float *out, int32_t *status) {
+    // A stand-in workspace, never dereferenced: every check but the workspace's runs, and
+    // nothing is launched.
+    return decode_impl(q, k_cache, v_cache, seq_lens, B, H_q, H_kv, d, L_max, 0, scale, dtype,
+                       out, reinterpret_cast<void *>(static_cast<uintptr_t>(256)), SIZE_MAX, status,
+                       nullptr, PagedArgs(), 1, nullptr, nullptr, true);
+}
+
 extern "C" int gqa_decode(const void *q, const void *k_cache, const void *v_cache,
                           const int32_t *seq_lens, int B, int H_q, int H_kv, int d, int L_max,
                           float scale, gqa_dtype_t dtype, float *out, void *workspace,
                           size_t workspace_bytes, int32_t *status, cudaStream_t stream) {
     return decode_impl(q, k_cache, v_cache, seq_lens, B, H_q, H_kv, d, L_max, 0, scale, dtype,
                        out, workspace, workspace_bytes, status, stream);
+}
+
+extern "C" int gqa_kv_append_decode(const void *q, const void *k_new, const void *v_new,
+                                    void *k_cache, void *v_cache, const int32_t *seq_lens,
+                                    int32_t *seq_lens_out, int B, int H_q, int H_kv, int d,
+                                    int L_max, float scale, gqa_dtype_t dtype, float *out,
+                                    void *workspace, size_t workspace_bytes, int32_t *status,
+                                    cudaStream_t stream) {
+    if (!k_new || !v_new || !seq_lens_out) return GQA_ERR_NULL;
+    if (dtype != GQA_DTYPE_BF16) return GQA_ERR_UNSUPPORTED_DTYPE;
+    if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(seq_lens_out, 4))
+        return GQA_ERR_ALIGNMENT;
+    if (B > 0 && seq_lens != nullptr) {
+        const uintptr_t a0 = reinterpret_cast<uintptr_t>(seq_lens), b0 = reinterpret_cast<uintptr_t>(seq_lens_out);
+        const uintptr_t n = static_cast<uintptr_t>(B) * sizeof(int32_t);
+        if (a0 < b0 + n && b0 < a0 + n) return GQA_ERR_OVERLAP;
+    }
+    AppendArgs ap;
+    ap.k_new = k_new;
+    ap.v_new = v_new;
+    ap.k_cache = k_cache;
+    ap.v_cache = v_cache;
+    ap.lens_out = seq_lens_out;
+    return decode_impl(q, k_cache, v_cache, seq_lens, B, H_q, H_kv, d, L_max, 0, scale, dtype, out,
+                       workspace, workspace_bytes, status, stream, PagedArgs(), 1, nullptr, nullptr,
+                       false, ap);
 }
 
 extern "C" int gqa_kv_append_paged(const void *k_new, const void *v_new, void *k_pool,
@@ -512,6 +565,7 @@ extern "C" const char *gqa_status_string(int code) {
         case GQA_ERR_CUDA: return "a CUDA runtime call failed";
         case GQA_ERR_NO_DEVICE: return "no usable sm_100 device is current";
         case GQA_ERR_SCRATCH_LIMIT: return "sizes need more scratch than the library's fixed no-allocation array";
+        case GQA_ERR_OVERLAP: return "the input and output length arrays overlap";
         default: return "unknown status code";
     }
 }

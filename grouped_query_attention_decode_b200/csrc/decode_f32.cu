@@ -48,8 +48,7 @@ split_f32_kernel(const float *__restrict__ q, const float *__restrict__ kc,
 
     grid_dependency_wait();
     if (warp == 0) {
-        long long *hdr = blockIdx.x == 0 ? reinterpret_cast<long long *>(p.ws) : nullptr;
-        const CtaRange cr = locate_cta_range(p, blockIdx.x, lane, hdr, blockIdx.x == 0);
+        const CtaRange cr = locate_cta_range(p, blockIdx.x, lane, blockIdx.x == 0);
         if (lane == 0) {
             s_begin = cr.begin;
             s_end = cr.end;
@@ -184,7 +183,7 @@ split_f32_kernel(const float *__restrict__ q, const float *__restrict__ kc,
                 }
             }
         } else {
-            float *slot = p.ws + p.hdr_floats + (static_cast<long long>(blockIdx.x) + sg.unit) * p.slot_floats;
+            float *slot = p.ws + p.slot_base + (static_cast<long long>(blockIdx.x) + sg.unit) * p.slot_floats;
 #pragma unroll
             for (int k = 0; k < ACC; ++k) {
                 const int idx = tid + 256 * k;

@@ -67,6 +67,7 @@ struct TcCfg {
 
     struct Small {
         uint64_t kv_full[8], kv_empty[8];
+        uint64_t ap_full[8];    // fused append: the copy of a tile that holds the appended row
         uint64_t q_full[2], q_empty[2];
         uint64_t s_full[2], s_empty[2], p_full[2], o_full[2], o_empty[2];
         uint64_t mma_done;
@@ -82,9 +83,17 @@ struct TcCfg {
     };
 
     static constexpr int SMEM_LIMIT = 232448;
-    static constexpr int BASE = 2 * P_BYTES + static_cast<int>(sizeof(Small));
-    // two q buffers (the next unit's q loads during the current unit) when two stages still fit
-    static constexpr int QB = (SMEM_LIMIT - BASE - 2 * Q_BYTES >= 2 * STAGE_BYTES) ? 2 : 1;
+    // Ring stages that fit next to pb P^T buffers and qb q buffers.
+    static constexpr int fit(int pb, int qb) {
+        return (SMEM_LIMIT - pb * P_BYTES - static_cast<int>(sizeof(Small)) - qb * Q_BYTES) / STAGE_BYTES;
+    }
+    // Two P^T buffers let the softmax write tile i's P while the tensor cores still read tile
+    // i-1's; one buffer (the softmax then waits for the previous P.V before it writes P) when
+    // that is what buys the ring a third stage.  Two q buffers (the next unit's q loads during
+    // the current unit) when two stages still fit.
+    static constexpr int PB = (fit(2, 2) < 3 && fit(1, 2) >= 3) ? 1 : 2;
+    static constexpr int QB = fit(PB, 2) >= 2 ? 2 : 1;
+    static constexpr int BASE = PB * P_BYTES + static_cast<int>(sizeof(Small));
     static constexpr int FIXED = BASE + QB * Q_BYTES;
     static constexpr int S_FIT = (SMEM_LIMIT - FIXED) / STAGE_BYTES;
     static constexpr int S = S_FIT > 6 ? 6 : S_FIT;
@@ -129,6 +138,126 @@ __device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t bytes) {
     return desc + static_cast<uint64_t>(bytes >> 4);
 }
 
+// The ticket warp under a fused append (gqa_kv_append_decode).  Besides the partial pieces'
+// tickets (run_ticket_warp), it owns the appended rows: for every tile that holds a unit's row
+// n - 1, it writes the new K and V rows (k_new, v_new) to the cache for later steps and, once
+// the tile's TMA copy has landed (that copy completes on ap_full instead of kv_full), over the
+// row the copy brought into the ring stage; then it completes the stage's kv_full itself, which
+// releases the tile to the tensor cores and the softmax warps as for any other tile.  The copy
+// may read the row before or after the cache write; nothing else in the kernel reads it.  An
+// event loop serves whichever of the next row and the next ticket is ready first.  Returns
+// false when a wait ran out.
+template <int D, int NG, int S, int STAGE_BYTES, int TILE_BYTES>
+__device__ bool append_ticket_warp(const DecodeParams &p, const CtaRange &cr, uint8_t *st_base,
+                                   uint64_t *kv_full, uint64_t *ap_full, uint64_t (*pc_full)[2],
+                                   uint64_t (*tk_done)[2], int (*tk_last)[2], int lane,
+                                   const volatile int *abort_flag, uint64_t budget) {
+    constexpr int T = 128;
+    constexpr int CH = D / 8;  // 16-byte chunks of a cached row of one head
+    // row cursor: the next tile that holds an appended row
+    SegmentWalker wr;
+    wr.init(p, cr);
+    Segment sr;
+    int tile_r = 0;  // walk index of the next segment's first tile
+    bool row_more = false, row_loaded = false;
+    int rt = 0, rrow = 0;  // walk index of the tile, the row within it
+    uint4 chunk = make_uint4(0, 0, 0, 0);
+    auto next_row = [&]() {
+        row_more = false;
+        row_loaded = false;
+        while (wr.next(sr)) {
+            const int first = tile_r;
+            tile_r += sr.len;
+            if (sr.appended && sr.j0 + sr.len == sr.nt) {
+                rt = first + sr.len - 1;
+                rrow = (sr.n - 1) - (sr.first + (sr.nt - 1) * T);
+                row_more = true;
+                return;
+            }
+        }
+    };
+    next_row();
+    // ticket cursor: the CTA's partial pieces (at most two), group by group
+    SegmentWalker wt;
+    wt.init(p, cr);
+    Segment stk;
+    int k = 0, g = 0;
+    bool tk_more = false;
+    auto next_piece = [&]() {
+        tk_more = false;
+        while (k < 2 && wt.next(stk))
+            if (!stk.whole) {
+                tk_more = true;
+                return;
+            }
+    };
+    next_piece();
+    const bool mine = lane < 2 * CH;
+    const int half = lane / CH, c = lane % CH;
+    // Per stage, the parity of its next ap_full phase: a stage's patched copies complete in
+    // order, and the producer issues the next one only after this warp released the previous
+    // (kv_full -> S.K^T -> P.V -> kv_empty), so the phases never run ahead of this warp.
+    uint32_t ap_phase = 0;
+    uint64_t idle_since = global_timer_ns();
+    uint32_t idle_polls = 0;
+    while (row_more || tk_more) {
+        bool progress = false;
+        if (row_more) {
+            if (!row_loaded) {
+                // the new row: one 16-byte chunk of K (lanes < CH) or V (the next CH lanes) per
+                // lane, written to the cache at once
+                if (mine) {
+                    const long long src = (static_cast<long long>(sr.b) * p.H_kv + sr.kvh) * CH + c;
+                    chunk = __ldg(static_cast<const uint4 *>(half ? p.v_new : p.k_new) + src);
+                    const long long dst = ((static_cast<long long>(sr.b) * p.L_max + (sr.n - 1)) * p.H_kv + sr.kvh) * CH + c;
+                    static_cast<uint4 *>(half ? p.v_cache : p.k_cache)[dst] = chunk;
+                }
+                row_loaded = true;
+            }
+            const int st = rt % S;
+            bool landed = lane == 0 ? mbar_test_wait(&ap_full[st], (ap_phase >> st) & 1u) : false;
+            if (__shfl_sync(kFullMask, landed, 0)) {
+                ap_phase ^= 1u << st;
+                if (mine) {
+                    // row rrow of the stage's K or V tile: 64-column blocks of T rows of 128 bytes,
+                    // the 16-byte chunks of a row XOR-swizzled by the row's low three bits
+                    uint8_t *base = st_base + st * STAGE_BYTES + half * TILE_BYTES;
+                    const int kb = c >> 3, cc = c & 7;
+                    *reinterpret_cast<uint4 *>(base + kb * T * 128 + rrow * 128 + ((cc ^ (rrow & 7)) << 4)) = chunk;
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&kv_full[st]);
+                next_row();
+                progress = true;
+            }
+        }
+        if (tk_more) {
+            bool done = lane == 0 ? mbar_test_wait(&pc_full[g][k], 0) : false;
+            if (__shfl_sync(kFullMask, done, 0)) {
+                if (lane == 0) {
+                    int c0, c1;
+                    tk_last[g][k] = take_ticket(p, stk.unit, g) == unit_pieces(stk.uoff, stk.nt, cr.total, p.G, c0, c1) - 1;
+                    mbar_arrive(&tk_done[g][k]);
+                }
+                if (++g == NG) {
+                    g = 0;
+                    ++k;
+                    next_piece();
+                }
+                progress = true;
+            }
+        }
+        if (progress) {
+            idle_polls = 0;
+        } else if ((++idle_polls & 15u) == 0) {
+            if (idle_polls == 16) idle_since = global_timer_ns();
+            if (*abort_flag || global_timer_ns() - idle_since > budget) return false;
+        }
+    }
+    return true;
+}
+
 template <int D, int NH, bool PAGED>
 __global__ void __launch_bounds__(TcCfg<D, NH>::THREADS, 1)
 split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -142,7 +271,7 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     uint8_t *const st_base = smem;
     uint8_t *const q_base = smem + S * C::STAGE_BYTES;
     uint8_t *const p_base = q_base + C::QB * C::Q_BYTES;
-    auto *const sm = reinterpret_cast<typename C::Small *>(p_base + 2 * C::P_BYTES);
+    auto *const sm = reinterpret_cast<typename C::Small *>(p_base + C::PB * C::P_BYTES);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -156,6 +285,7 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int s = 0; s < S; ++s) {
             mbar_init(&sm->kv_full[s], 1);
             mbar_init(&sm->kv_empty[s], 1);
+            mbar_init(&sm->ap_full[s], 1);
         }
         for (int j = 0; j < 2; ++j) {
             mbar_init(&sm->q_full[j], 1);
@@ -194,8 +324,7 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // Everything below reads what the previous kernel on the stream (the append) wrote.
     grid_dependency_wait();
     if (warp == 2) {
-        long long *hdr = blockIdx.x == 0 ? reinterpret_cast<long long *>(p.ws) : nullptr;
-        const CtaRange cr = locate_cta_range(p, blockIdx.x, lane, hdr, blockIdx.x == 0);
+        const CtaRange cr = locate_cta_range(p, blockIdx.x, lane, blockIdx.x == 0);
         if (lane == 0) {
             sm->begin = cr.begin;
             sm->end = cr.end;
@@ -240,6 +369,7 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         Segment sg;
         int i = 0, sidx = 0;
         bool ok = true;
+        uint32_t ap_mask = 0, ap_par = 0;  // fused append: stages whose copy lands on ap_full
         [[maybe_unused]] TileCursor ahead;
         [[maybe_unused]] int pg_ring[kPageAhead];
         if constexpr (PAGED) {
@@ -289,6 +419,15 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 uint8_t *kdst = st_base + st * C::STAGE_BYTES;
                 uint8_t *vdst = kdst + C::TILE_BYTES;
+                // A tile that holds a fused append's row lands on ap_full; the ticket warp writes
+                // the row over the copy and then completes kv_full itself.
+                uint64_t *full = &sm->kv_full[st];
+                ap_mask &= ~(1u << st);
+                if (!PAGED && sg.appended && sg.j0 + sg.len == sg.nt && jj == sg.len - 1) {
+                    full = &sm->ap_full[st];
+                    ap_mask |= 1u << st;   // the copy now in flight in stage st lands on ap_full
+                    ap_par ^= 1u << st;    // with the phase parity before this flip
+                }
                 if constexpr (PAGED) {
                     // boxes of min(page_size, T) rows, or 8 rows for a partial tile
                     const int boxr = rows == T ? min(p.page_size, T) : 8;
@@ -311,20 +450,20 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     }
                 } else if (lane == 0) {
                     if (rows == T) {
-                        mbar_arrive_expect_tx(&sm->kv_full[st], C::STAGE_BYTES);
+                        mbar_arrive_expect_tx(full, C::STAGE_BYTES);
 #pragma unroll
                         for (int kb = 0; kb < C::KB; ++kb) {
-                            tma_load_4d(kdst + kb * T * 128, &tm_k, &sm->kv_full[st], kb * 64, sg.kvh, row0, sg.b, pol);
-                            tma_load_4d(vdst + kb * T * 128, &tm_v, &sm->kv_full[st], kb * 64, sg.kvh, row0, sg.b, pol);
+                            tma_load_4d(kdst + kb * T * 128, &tm_k, full, kb * 64, sg.kvh, row0, sg.b, pol);
+                            tma_load_4d(vdst + kb * T * 128, &tm_v, full, kb * 64, sg.kvh, row0, sg.b, pol);
                         }
                     } else {
                         const int nb = (rows + 7) >> 3;  // 8-row boxes: at most 7 rows past n
-                        mbar_arrive_expect_tx(&sm->kv_full[st], 2 * C::KB * nb * 8 * 128);
+                        mbar_arrive_expect_tx(full, 2 * C::KB * nb * 8 * 128);
                         for (int x = 0; x < nb; ++x) {
 #pragma unroll
                             for (int kb = 0; kb < C::KB; ++kb) {
-                                tma_load_4d(kdst + kb * T * 128 + x * 1024, &tm_k8, &sm->kv_full[st], kb * 64, sg.kvh, row0 + 8 * x, sg.b, pol);
-                                tma_load_4d(vdst + kb * T * 128 + x * 1024, &tm_v8, &sm->kv_full[st], kb * 64, sg.kvh, row0 + 8 * x, sg.b, pol);
+                                tma_load_4d(kdst + kb * T * 128 + x * 1024, &tm_k8, full, kb * 64, sg.kvh, row0 + 8 * x, sg.b, pol);
+                                tma_load_4d(vdst + kb * T * 128 + x * 1024, &tm_v8, full, kb * 64, sg.kvh, row0 + 8 * x, sg.b, pol);
                             }
                         }
                     }
@@ -334,9 +473,15 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         if (lane == 0) {
             if (!ok) fail();
-            // Drain: no copy may still be writing this CTA's shared memory when it exits.
-            for (int ii = (i > S ? i - S : 0); ii < i; ++ii)
-                wait_bounded(&sm->kv_full[ii % S], (ii / S) & 1, nullptr, kDrainNs);
+            // Drain: no copy may still be writing this CTA's shared memory when it exits (a
+            // patched tile's copy completes on ap_full, which the ticket warp waits for).
+            for (int ii = (i > S ? i - S : 0); ii < i; ++ii) {
+                const int st = ii % S;
+                if (ap_mask & (1u << st))
+                    wait_bounded(&sm->ap_full[st], ((ap_par >> st) & 1u) ^ 1u, nullptr, kDrainNs);
+                else
+                    wait_bounded(&sm->kv_full[st], (ii / S) & 1, nullptr, kDrainNs);
+            }
             for (int ss = (sidx > C::QB ? sidx - C::QB : 0); ss < sidx; ++ss)
                 wait_bounded(&sm->q_full[ss % C::QB], (ss / C::QB) & 1, nullptr, kDrainNs);
         }
@@ -400,7 +545,7 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         (pv_t < 2 || mbar_test_wait(&sm->o_empty[j2], ((pv_t >> 1) - 1) & 1))) {
                         tc_fence_after_sync();
                         const uint64_t dv = desc_add(dv0, (pv_t % S) * C::STAGE_BYTES);
-                        const uint64_t dp = desc_add(dp0, j2 * C::P_BYTES);
+                        const uint64_t dp = desc_add(dp0, (j2 % C::PB) * C::P_BYTES);
                         // O^T[:, 0:RP] = V^T.P_hi^T and O^T[:, RP:2RP] = V^T.P_lo^T in one
                         // N = 2*RP product.
 #pragma unroll
@@ -430,7 +575,15 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
     } else if (warp == C::TICKET_WARP) {
         // ------------------------------------------------------------------ ticket warp
-        run_ticket_warp<C::NWG>(p, cr, sm->pc_full, sm->tk_done, sm->tk_last, lane, abort_flag, budget);
+        if (!PAGED && p.append) {
+            if (!append_ticket_warp<D, C::NWG, S, C::STAGE_BYTES, C::TILE_BYTES>(
+                    p, cr, st_base, sm->kv_full, sm->ap_full, sm->pc_full, sm->tk_done, sm->tk_last, lane,
+                    abort_flag, budget) &&
+                lane == 0)
+                fail();
+        } else {
+            run_ticket_warp<C::NWG>(p, cr, sm->pc_full, sm->tk_done, sm->tk_last, lane, abort_flag, budget);
+        }
     } else {
         // ------------------------------------------------------------------ softmax warps
         // NWG warpgroups of four warps; warpgroup g owns query heads [g*NHW, (g+1)*NHW) of the
@@ -563,7 +716,7 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 // `row` of the MN-major P^T: high parts at values [0, RP), low parts at
                 // [RP, 2RP), written as 16-byte chunks of 8 heads.
                 {
-                    uint8_t *prow = p_base + j2 * C::P_BYTES + row * C::P_ROWB;
+                    uint8_t *prow = p_base + (j2 % C::PB) * C::P_BYTES + row * C::P_ROWB;
                     const int swz = C::P_ROWB == 128 ? (row & 7) : ((row >> 1) & 3);
                     constexpr int HALF_VALS = C::P_ROWB / 2;  // bf16 values per atom row
 #pragma unroll
@@ -573,6 +726,11 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         x[h] = x[h] == -INFINITY ? 0.f : ex2_approx(x[h] - m_run[h]);
                         l[h] = l[h] * alpha[h] + x[h];
                     }
+                    // One P^T buffer: the previous tile's P.V must have read it (its O is folded
+                    // below, after this tile's P is handed over).
+                    if (C::PB == 1 && jj > 0 && !bad &&
+                        !wait_bounded(&sm->o_full[(i - 1) & 1], ((i - 1) >> 1) & 1, abort_flag, budget))
+                        bad = true;
 #pragma unroll
                     for (int c8 = 0; c8 < (NHW + 7) / 8; ++c8) {
                         uint32_t hw[4], lw[4];
@@ -667,7 +825,7 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     }
                 } else {
                     // slot: O [RB][D], then m [RB], then l [RB] (padding columns included)
-                    float *slot = p.ws + p.hdr_floats +
+                    float *slot = p.ws + p.slot_base +
                                   (static_cast<long long>(blockIdx.x) + sg.unit) * p.slot_floats;
 #pragma unroll
                     for (int h = 0; h < NHW; ++h)

@@ -230,8 +230,7 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     // Everything below reads what the previous kernel on the stream (the append) wrote.
     grid_dependency_wait();
     if (warp == 2) {
-        long long *hdr = blockIdx.x == 0 ? reinterpret_cast<long long *>(p.ws) : nullptr;
-        const CtaRange cr = locate_cta_range(p, blockIdx.x, lane, hdr, blockIdx.x == 0);
+        const CtaRange cr = locate_cta_range(p, blockIdx.x, lane, blockIdx.x == 0);
         if (lane == 0) {
             sm->begin = cr.begin;
             sm->end = cr.end;
@@ -763,7 +762,7 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                         if (orow >= 0) p.out[orow * D + dcol] = O[h] * vs / Lh[h];
                     }
                 } else {
-                    float *slot = p.ws + p.hdr_floats +
+                    float *slot = p.ws + p.slot_base +
                                   (static_cast<long long>(blockIdx.x) + sg.unit) * p.slot_floats;
 #pragma unroll
                     for (int h = 0; h < NHW; ++h)

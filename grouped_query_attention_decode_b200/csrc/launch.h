@@ -6,6 +6,8 @@
 
 #include <cstdint>
 
+#include "gqa.h"
+
 namespace gqa {
 
 struct DecodeParams;
@@ -26,6 +28,11 @@ int tc8_tile_rows(int heads_per_unit);
 // Byte offset and size of the per-unit piece counters inside a decode workspace for these
 // sizes on the current device (0 bytes when the sizes are invalid).
 size_t decode_counter_region(int B, int H_q, int H_kv, int d, size_t *offset);
+// Every host-side check gqa_decode makes except those of the workspace, in the same order and
+// with the same return codes; launches nothing.
+int decode_check(const void *q, const void *k_cache, const void *v_cache, const int32_t *seq_lens,
+                 int B, int H_q, int H_kv, int d, int L_max, float scale, gqa_dtype_t dtype,
+                 float *out, int32_t *status);
 int launch_split_tc8(const TmaMaps &maps, const void *q, const DecodeParams &p, cudaStream_t stream);
 int launch_append_fp8(const void *k_new, const void *v_new, bool bf16_in, void *k_cache,
                       void *v_cache, const float *k_scale, const float *v_scale, int32_t *seq_lens,

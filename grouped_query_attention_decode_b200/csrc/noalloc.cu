@@ -52,19 +52,16 @@ extern "C" int gqa_decode_noalloc(const void *q, const void *k_cache, const void
                                   int L_max, float scale, gqa_dtype_t dtype, float *out,
                                   int32_t *status, cudaStream_t stream) {
     const size_t need = gqa_decode_workspace_size(B, H_q, H_kv, d, dtype);
-    if (need == 0) {
-        // invalid sizes or no device: let gqa_decode report which
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess) {
-            cudaGetLastError();
-            return GQA_ERR_NO_DEVICE;
-        }
-        return gqa_decode(q, k_cache, v_cache, seq_lens, B, H_q, H_kv, d, L_max, scale, dtype,
-                          out, nullptr, 0, status, stream);
-    }
     if (need > kScratchBytes) return GQA_ERR_SCRATCH_LIMIT;
+    // Every other host-side check of gqa_decode (pointers, alignment, sizes, element type,
+    // scale, device), before anything is queued on the stream; need == 0 (invalid sizes or no
+    // usable device) is reported here with gqa_decode's own code.
+    int rc = gqa::decode_check(q, k_cache, v_cache, seq_lens, B, H_q, H_kv, d, L_max, scale,
+                               dtype, out, status);
+    if (rc != GQA_OK) return rc;
+    if (need == 0) return GQA_ERR_SHAPE;  // not reached: decode_check refuses those sizes
     void *ws = nullptr;
-    const int rc = scratch_address(&ws);
+    rc = scratch_address(&ws);
     if (rc != GQA_OK) return rc;
     // The workspace's piece counters must be zero; a call that timed out may have left some
     // set, and the caller cannot reach this array, so clear them on the stream every time.

@@ -23,7 +23,7 @@ namespace gqa {
 struct DecodeParams {
     const int32_t *seq_lens;  // [B] rows attended per sequence
     float *out;               // [B][H_q][d]
-    float *ws;                // workspace: int64 header, then partial slots
+    float *ws;                // workspace: per-unit piece counters, then partial slots
     int32_t *status;          // device status word or nullptr
     int B, H_q, H_kv, d, L_max;
     int r;     // query heads per key/value head
@@ -44,11 +44,18 @@ struct DecodeParams {
     // FP8 (e4m3) cache: a code of key/value head g stands for value(code) * k_scale[g] (K)
     // or value(code) * v_scale[g] (V); nullptr for 16- and 32-bit caches.
     const float *k_scale, *v_scale;
+    // Append fused into the decode (gqa_kv_append_decode): k_new / v_new [B][H_kv][d] go to row
+    // seq_lens[b] of the cache, which the decode then attends (n_b = seq_lens[b] + 1); the
+    // lengths after the append are written to lens_out (never to seq_lens).  append = 0: none.
+    const void *k_new, *v_new;
+    void *k_cache, *v_cache;  // [B][L_max][H_kv][d], for the appended rows
+    int32_t *lens_out;
+    int append;
     int32_t *cnt;                     // [units] pieces of each unit finished in this call (0 between calls)
     float scale_log2;                 // softmax scale * log2(e)
     unsigned long long wait_ns;       // bound of every pipeline wait
     long long slot_floats;            // RB * (d + 2) rounded up to a multiple of 4
-    long long hdr_floats;             // header length in floats (int64 offsets [B + 1])
+    long long slot_base;              // offset of the first partial slot in ws, in floats
 };
 
 // Row of out [B*Q][H_q] that unit column hh (token hh / rb, head hh % rb) writes, or -1 for a
@@ -67,6 +74,18 @@ __device__ __forceinline__ int valid_len(int n, int L_max, int Q) {
 }
 
 __device__ __forceinline__ int tiles_of(int n, int T) { return (n + T - 1) / T; }
+
+// Does a fused append take place for a sequence whose length before it is `raw`?  Only when
+// the row fits: 0 <= raw < L_max (gqa_kv_append refuses the others the same way).
+__device__ __forceinline__ bool append_fits(int raw, int L_max) { return raw >= 0 && raw < L_max; }
+
+// Rows sequence b is asked to attend: seq_lens[b], plus the appended row under a fused append.
+__device__ __forceinline__ int asked_len(const DecodeParams &p, int b, bool *appended = nullptr) {
+    const int raw = p.seq_lens[b];
+    const bool app = p.append && append_fits(raw, p.L_max);
+    if (appended != nullptr) *appended = app;
+    return app ? raw + 1 : raw;
+}
 
 // First attended row of a sequence with n rows: n - window under a sliding window, else 0.
 __device__ __forceinline__ int first_row(int n, int window) {
@@ -104,28 +123,29 @@ struct CtaRange {
     long long offl;  // first tile of sequence bl on the line
 };
 
-// Whole warp: total tiles, this CTA's range and where it starts.  When `hdr` is not null the
-// warp also stores the exclusive prefix of tiles per sequence (hdr[b], b <= B; hdr[B] = total).
-// When `flag_range` is set, lengths outside [0, L_max] set GQA_STATUS_SEQLEN_RANGE.
-__device__ inline CtaRange locate_cta_range(const DecodeParams &p, int cta, int lane, long long *hdr,
-                                     bool flag_range) {
+// Whole warp: total tiles, this CTA's range and where it starts.  When `flag_range` is set,
+// lengths outside [0, L_max] set GQA_STATUS_SEQLEN_RANGE.
+__device__ inline CtaRange locate_cta_range(const DecodeParams &p, int cta, int lane, bool flag_range) {
     long long run = 0;
     for (int base = 0; base < p.B; base += 32) {
         const int b = base + lane;
         int n = 0;
         if (b < p.B) {
-            const int raw = p.seq_lens[b];
-            n = valid_len(raw, p.L_max, p.Q);
-            if (flag_range && n != raw && p.status != nullptr) atomicOr(p.status, GQA_STATUS_SEQLEN_RANGE);
+            bool app = false;
+            const int asked = asked_len(p, b, &app);
+            n = valid_len(asked, p.L_max, p.Q);
+            if (flag_range) {
+                if (n != asked && p.status != nullptr) atomicOr(p.status, GQA_STATUS_SEQLEN_RANGE);
+                if (p.append && !app && p.status != nullptr) atomicOr(p.status, GQA_STATUS_APPEND_OVERFLOW);
+                if (p.append) p.lens_out[b] = asked;
+            }
         }
         const long long v = static_cast<long long>(seq_tiles(n, p)) * p.UB;
         const long long incl = warp_incl_scan(v, lane);
-        if (hdr != nullptr && b < p.B) hdr[b] = run + incl - v;
         run += __shfl_sync(kFullMask, incl, 31);
     }
     CtaRange cr;
     cr.total = run;
-    if (hdr != nullptr && lane == 0) hdr[p.B] = run;
     cr.begin = cta_range_begin(cta, run, p.G);
     cr.end = cta_range_begin(cta + 1, run, p.G);
     cr.b0 = 0;
@@ -137,7 +157,7 @@ __device__ inline CtaRange locate_cta_range(const DecodeParams &p, int cta, int 
     bool found0 = false;
     for (int base = 0; base < p.B; base += 32) {
         const int b = base + lane;
-        const int n = b < p.B ? valid_len(p.seq_lens[b], p.L_max, p.Q) : 0;
+        const int n = b < p.B ? valid_len(asked_len(p, b), p.L_max, p.Q) : 0;
         const long long v = static_cast<long long>(seq_tiles(n, p)) * p.UB;
         const long long incl = warp_incl_scan(v, lane);
         const long long excl = incl - v;
@@ -168,6 +188,7 @@ struct Segment {
     int first;       // first attended row (0 unless a sliding window cuts the front)
     int unit;        // unit index b * UB + (kvh * HB + hb)
     bool whole;      // the piece is the entire unit
+    bool appended;   // a fused append writes row n - 1 of the sequence
     int nt;          // tiles of the unit
     long long uoff;  // line position of the unit's first tile
 };
@@ -179,12 +200,21 @@ struct Segment {
 // walker; all of them see the same sequence of segments.
 struct SegmentWalker {
     const int32_t *lens;
-    int B, UB, HB, L_max, T, window, Q;
+    int B, UB, HB, L_max, T, window, Q, append;
     int b, n, nt;
+    bool app;         // sequence b takes a fused append
     long long off, t, end;
     bool last_first;  // the range's last segment is still to be returned first
     int bl, nl, ntl, kl;
+    bool appl;
     long long offl, tl, endl;
+
+    // Rows sequence bb attends (and whether a fused append writes its last one).
+    __device__ int rows_of(int bb, bool &a) const {
+        const int raw = lens[bb];
+        a = append && append_fits(raw, L_max);
+        return valid_len(a ? raw + 1 : raw, L_max, Q);
+    }
 
     __device__ void init(const DecodeParams &p, const CtaRange &cr) {
         lens = p.seq_lens;
@@ -195,17 +225,19 @@ struct SegmentWalker {
         T = p.T;
         window = p.window;
         Q = p.Q;
+        append = p.append;
         t = cr.begin;
         end = cr.end;
         b = cr.b0;
         off = cr.off0;
         last_first = false;
+        app = appl = false;
         if (t < end) {
-            n = valid_len(lens[b], L_max, Q);
+            n = rows_of(b, app);
             nt = tiles_of(n - first_row(n, window), T);
             bl = cr.bl;
             offl = cr.offl;
-            nl = valid_len(lens[bl], L_max, Q);
+            nl = rows_of(bl, appl);
             ntl = tiles_of(nl - first_row(nl, window), T);
             kl = static_cast<int>((end - 1 - offl) / ntl);
             const long long uoffl = offl + static_cast<long long>(kl) * ntl;
@@ -236,6 +268,7 @@ struct SegmentWalker {
             s.nt = ntl;
             s.uoff = tl;
             s.whole = len == ntl;
+            s.appended = appl;
             return true;
         }
         if (t >= end) return false;
@@ -245,7 +278,7 @@ struct SegmentWalker {
                 t = end;
                 return false;
             }
-            n = valid_len(lens[b], L_max, Q);
+            n = rows_of(b, app);
             nt = tiles_of(n - first_row(n, window), T);
         }
         const long long rel = t - off;
@@ -264,6 +297,7 @@ struct SegmentWalker {
         s.nt = nt;
         s.uoff = off + static_cast<long long>(k) * nt;
         s.whole = (j0 == 0 && len == nt);
+        s.appended = app;
         t += len;
         return true;
     }
@@ -326,7 +360,7 @@ __device__ inline void merge_unit(const DecodeParams &p, const PendingPiece &u, 
     unit_pieces(u.uoff, u.nt, total, p.G, c0, c1);
     const int nh = p.RB, d = p.d;
     h1 = min(h1, nh);
-    const float *base = p.ws + p.hdr_floats + static_cast<long long>(u.unit) * p.slot_floats;
+    const float *base = p.ws + p.slot_base + static_cast<long long>(u.unit) * p.slot_floats;
     const bool some_empty = total < p.G;
     const int nvec = (h1 - h0) * d / 4;
     // The non-empty pieces c0 .. c1 in line order (a CTA with an empty range holds none).
@@ -498,7 +532,7 @@ __device__ inline void zero_empty_units(const DecodeParams &p, int cta, int tid,
     const int units = p.B * p.UB;
     for (int u = cta; u < units; u += p.G) {
         const int b = u / p.UB;
-        if (seq_tiles(valid_len(p.seq_lens[b], p.L_max, p.Q), p) != 0) continue;
+        if (seq_tiles(valid_len(asked_len(p, b), p.L_max, p.Q), p) != 0) continue;
         const int k = u - b * p.UB;
         const int kvh = k / p.HB, hb = k - kvh * p.HB;
         for (int idx = tid; idx < p.RB * p.d; idx += nthr) {

@@ -70,6 +70,8 @@ typedef enum {
 #define GQA_ERR_NO_DEVICE (-9)            /* no usable sm_100 device is current */
 #define GQA_ERR_SCRATCH_LIMIT (-10)       /* gqa_decode_noalloc: the sizes need more scratch than
                                              GQA_NOALLOC_SCRATCH_BYTES */
+#define GQA_ERR_OVERLAP (-11)             /* gqa_kv_append_decode: seq_lens and seq_lens_out
+                                             overlap */
 
 /* Device-side status bits (OR-ed into *status). */
 #define GQA_STATUS_APPEND_OVERFLOW 1  /* gqa_kv_append: seq_lens[b] < 0 or >= L_max; row skipped */
@@ -138,6 +140,31 @@ int gqa_decode(const void *q, const void *k_cache, const void *v_cache, const in
                int B, int H_q, int H_kv, int d, int L_max, float scale, gqa_dtype_t dtype,
                float *out, void *workspace, size_t workspace_bytes, int32_t *status,
                cudaStream_t stream);
+
+/*
+ * gqa_kv_append_decode: the whole of Algorithm 2 of "GQA 阅读笔记" (append, then attend over the
+ * t + 1 rows) in ONE kernel launch: the result of gqa_kv_append followed by gqa_decode, bit for
+ * bit, with the lengths kept in two arrays instead of incremented in place.  With
+ * t = seq_lens[b] on entry:
+ *   - 0 <= t < L_max: k_new[b] / v_new[b] are written to row t of the caches (bit-exact), the
+ *     decode attends rows [0, t + 1), and seq_lens_out[b] = t + 1;
+ *   - otherwise the row is not written (GQA_STATUS_APPEND_OVERFLOW) and the decode attends t
+ *     rows as gqa_decode would (t = L_max: all of them; t < 0 or t > L_max: out[b] = 0 and
+ *     GQA_STATUS_SEQLEN_RANGE); seq_lens_out[b] = t.
+ * seq_lens is only read (every CTA of the kernel reads it, so it cannot change during the
+ * call); seq_lens_out [B] int32 device is only written, and the two must not overlap
+ * (GQA_ERR_OVERLAP).  A decode loop passes the two arrays alternately.  Only one CTA of the
+ * kernel writes each appended row, just before that row's tile is copied for the decode, so
+ * the row reaches the cache and the attention in the same pass; no other row of the cache is
+ * written.  bfloat16 only (GQA_ERR_UNSUPPORTED_DTYPE otherwise); the workspace is that of
+ * gqa_decode (gqa_decode_workspace_size), with the same zero-fill rule.  Other arguments, layouts
+ * and errors as gqa_kv_append and gqa_decode.
+ */
+int gqa_kv_append_decode(const void *q, const void *k_new, const void *v_new, void *k_cache,
+                         void *v_cache, const int32_t *seq_lens, int32_t *seq_lens_out, int B,
+                         int H_q, int H_kv, int d, int L_max, float scale, gqa_dtype_t dtype,
+                         float *out, void *workspace, size_t workspace_bytes, int32_t *status,
+                         cudaStream_t stream);
 
 /*
  * gqa_decode_window: gqa_decode with a sliding window.  Each query head of sequence b attends
@@ -268,6 +295,9 @@ int gqa_decode_paged_fp8(const void *q, const void *k_pool, const void *v_pool,
  *
  *   - Sizes whose gqa_decode_workspace_size() exceeds GQA_NOALLOC_SCRATCH_BYTES are refused
  *     with GQA_ERR_SCRATCH_LIMIT before anything runs (use gqa_decode with a workspace).
+ *   - Every other host-side check of gqa_decode (pointers, alignment, sizes, element type,
+ *     scale, device) also runs before anything is queued on `stream`, with gqa_decode's
+ *     return codes.
  *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
  *     with that device current and caches it; make that first call before any stream capture.
  *   - Each call first clears the array's counters with one cudaMemsetAsync on `stream` (the

@@ -53,15 +53,5 @@ def max_err(out: torch.Tensor, ref: dict) -> float:
     return max(float(np.max(np.abs(o[b] - r))) for b, r in ref.items())
 
 
-def sample_bs(lengths, k_random=1, seed=0):
-    """A few sequences for full-size checks: first, last, shortest, longest and random ones."""
-    lens = [int(v) for v in lengths]
-    B = len(lens)
-    s = {0, B - 1, int(np.argmin(lens)), int(np.argmax(lens))}
-    rng = np.random.default_rng(seed)
-    s.update(int(v) for v in rng.integers(0, B, size=k_random))
-    return sorted(s)
-
-
 def workload(name):
     return inputs.WORKLOADS[name]

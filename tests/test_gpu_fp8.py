@@ -124,7 +124,7 @@ def test_fp8_decode_window(oracle, window):
 
 def test_fp8_full_size_llama(oracle):
     w = inputs.WORKLOADS["llama2_70b_layer_fp8"]
-    _step(oracle, w, bs=[0, 9, 15])
+    _step(oracle, w, bs=list(range(w.B)))
 
 
 @pytest.mark.parametrize("page_size", [8, 16, 64, 256, 512])

@@ -1,7 +1,7 @@
 """GPU parity: the CUDA path through the C ABI against the CPU oracle, element by element.
 
-Small cases are checked on every output; the full-size workloads (the shapes the benchmark
-times, launched the same way) on every output of a sample of sequences.  Tolerances: max abs
+Small cases and the full-size workloads (the shapes the benchmark times, launched the same
+way) are checked on every output.  Tolerances: max abs
 error 1e-5 for float32 inputs, 2e-3 for bf16 caches (fp32 accumulation; the oracle gets the
 same bf16-rounded values).  The append is checked bit for bit.  Cache rows past each sequence's
 length are NaN in these tests, so any read past the length shows up as NaN in the output.
@@ -10,7 +10,7 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_helpers import TOL, max_err, oracle_step, run_step, sample_bs, workload
+from gpu_helpers import TOL, max_err, oracle_step, run_step, workload
 from grouped_query_attention_decode_b200 import inputs
 
 pytestmark = pytest.mark.gpu
@@ -35,16 +35,18 @@ def test_tiny_fp32(oracle):
 @pytest.mark.parametrize("name", ["llama2_70b_layer", "t5xxl_g64_mha", "t5xxl_g8", "t5xxl_g1_mqa",
                                   "mqa_long", "ragged_long"])
 def test_full_size_workloads(oracle, name):
+    # every output of every sequence, at the sizes and in the launch configuration the
+    # benchmark times
     w = workload(name)
     x = inputs.make_inputs(w, poison=False)
-    bs = sample_bs(x["lengths"], k_random=2, seed=w.seed)
     out, lens, status, _ = run_step(x)
     assert status == 0, f"device status {status}"
     assert torch.equal(lens.cpu(), x["lengths"])
     assert torch.isfinite(out).all()
-    ref = oracle_step(oracle, x, bs)
+    ref = oracle_step(oracle, x, None)
+    assert len(ref) == w.B
     err = max_err(out, ref)
-    assert err <= TOL[w.dtype], f"{name}: max abs error {err} on sequences {bs}"
+    assert err <= TOL[w.dtype], f"{name}: max abs error {err}"
 
 
 # group sizes 1..128 (128 = two blocks of 64 query heads), both head dims, lengths spanning

@@ -3,7 +3,7 @@
 Such callers (a plugin whose host framework owns all device memory, a serving loop that must
 not call cudaMalloc and has no buffer to lend) get the library's own fixed scratch array.  This
 file checks, through the C ABI, that the allocation-free call returns what gqa_decode returns
-with a caller workspace, on two calls in a row (the second reuses the array the first left
+with a caller workspace (bit for bit: the same kernel runs), on two calls in a row (the second reuses the array the first left
 behind), and that sizes needing more scratch than the array holds are refused.  It sits last
 in collection order so that a failure here leaves every other test already run.
 """
@@ -13,7 +13,6 @@ import pytest
 import torch
 
 import grouped_query_attention_decode_b200 as gqa
-from gpu_helpers import TOL
 from grouped_query_attention_decode_b200 import inputs
 
 pytestmark = pytest.mark.gpu
@@ -58,9 +57,10 @@ def test_noalloc_matches_workspace_entry_point(w):
         outs.append(out)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
+    # the same kernel on the same inputs with a fixed merge order: identical bits
     for out in outs:
         assert torch.isfinite(out).all()
-        assert float((out - ref).abs().max()) <= TOL[w.dtype]
+        assert torch.equal(out, ref)
 
 
 def test_noalloc_refuses_sizes_beyond_its_array():
