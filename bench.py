@@ -47,6 +47,9 @@ DEFAULT_WORKLOAD = "llama2_70b_layer"
 ALSO_DEFAULT = "ragged_long"
 PROFILE_DIR = os.path.join(ROOT, "profiles")
 CSRC = os.path.join(ROOT, "grouped_query_attention_decode_b200", "csrc")
+# GPU-side spin (clock cycles, ~0.2 ms) that holds the stream while the host queues a timed
+# region's launches
+HOST_GATE_CYCLES = 400_000
 KERNEL_SOURCES = {
     "split_tc_kernel": ("decode_tc.cu", "device.cuh", "schedule.cuh"),
     "split_tc8_kernel": ("decode_tc8.cu", "device.cuh", "schedule.cuh"),
@@ -449,25 +452,33 @@ class Replica:
                     for j in range(n):
                         self.decode(j % self.n_copies, self.lens_dec)
                 else:
-                    rows.copy_(init)
+                    if not self.fused:  # the fused step only writes its length rows
+                        rows.copy_(init)
                     for j in range(n):
                         self.step(j % self.n_copies, rows[j])
         torch.cuda.current_stream().wait_stream(cap)
         torch.cuda.synchronize()
         return g, (rows, init)
 
-    def time_steps(self, K: int, W: int) -> float:
-        """Device time (ms) of exactly K steps after >= W untimed ones, on the current stream
-        between a synchronize and a synchronize."""
+    def time_steps(self, K: int, W: int, barrier=None) -> float:
+        """Device time (ms) of exactly K steps, on the current stream, with a barrier (all
+        ranks) and a synchronize before and after.  After the barrier, a GPU-side spin holds the
+        stream while the host queues W untimed warm-up steps, the first event, the K timed steps
+        and the last event: host launch latency stays outside the timed region, and the first
+        timed step follows a step on a busy GPU exactly as every later one does."""
         ng = self.n_copies * max(1, 64 // self.n_copies)
         full, keep_full = self._capture(ng)
         tail = K % ng
         tail_g, keep_tail = self._capture(tail) if tail else (None, None)
+        warm_g, keep_warm = self._capture(W)
         for _ in range(max(1, -(-W // ng))):
             full.replay()
+        (barrier or torch.cuda.synchronize)()
         torch.cuda.synchronize()
         stream = torch.cuda.current_stream()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda._sleep(HOST_GATE_CYCLES)
+        warm_g.replay()
         e0.record(stream)
         for _ in range(K // ng):
             full.replay()
@@ -475,8 +486,9 @@ class Replica:
             tail_g.replay()
         e1.record(stream)
         torch.cuda.synchronize()
+        (barrier or torch.cuda.synchronize)()
         assert int(self.status.item()) == 0, f"device status {int(self.status.item())}"
-        del full, tail_g, keep_full, keep_tail
+        del full, tail_g, warm_g, keep_full, keep_tail, keep_warm
         return e0.elapsed_time(e1)
 
     def time_kernel(self, min_launches: int, min_seconds: float) -> list[float]:
@@ -499,6 +511,7 @@ class Replica:
         reps = min(reps, max(5, 200000 // kg))
         stream = torch.cuda.current_stream()
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+        torch.cuda._sleep(HOST_GATE_CYCLES)
         ev[0].record(stream)
         for i in range(reps):
             g.replay()
@@ -617,9 +630,7 @@ def run_replica(args, rank, world, local, dev, pg, make_replica):
     # K timed steps
     barrier()
     launch_us = rep.time_kernel(args.kernel_launches, args.kernel_seconds)
-    barrier()
-    t_ms = rep.time_steps(K, W)
-    barrier()
+    t_ms = rep.time_steps(K, W, barrier)
     clk = clocks.stop()
     ms_step = max_over_ranks(t_ms / K, pg, dev)
     launch_us_max = max_over_ranks(statistics.mean(launch_us), pg, dev)
@@ -701,9 +712,7 @@ def time_also(args, rank, world, local, dev, pg, make_replica, peak, peak_kind, 
     clocks = ClockSampler(local, enabled=not args.no_clocks)
     barrier()
     launch_us = r2.time_kernel(args.kernel_launches, args.kernel_seconds)
-    barrier()
-    t_ms = r2.time_steps(args.steps, args.warmup)
-    barrier()
+    t_ms = r2.time_steps(args.steps, args.warmup, barrier)
     clk = clocks.stop()
     ms_step = max_over_ranks(t_ms / args.steps, pg, dev)
     value = r2.ideal * world / (ms_step * 1e-3) / 1e9

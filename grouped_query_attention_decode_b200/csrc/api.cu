@@ -55,11 +55,15 @@ struct Geometry {
 };
 
 // Units: (sequence, key/value head, block of rb query heads) with Q query tokens each; a unit
-// has RB = Q * rb <= 64 columns.
+// has RB = Q * rb <= kMaxUnitCols columns.  A group of more than 32 query heads is cut into
+// blocks of 32 that read the same K/V tiles (the second read of a tile finds it in L2 when the
+// blocks' pieces run close together), which keeps every softmax thread's per-column state in
+// registers.
+constexpr int kMaxUnitCols = 32;
 Geometry geometry(int B, int H_q, int H_kv, int d, int G, int Q = 1) {
     Geometry g;
     g.r = H_q / H_kv;
-    g.rb = g.r < 64 / Q ? g.r : 64 / Q;
+    g.rb = g.r < kMaxUnitCols / Q ? g.r : kMaxUnitCols / Q;
     g.RB = Q * g.rb;
     g.HB = (g.r + g.rb - 1) / g.rb;
     g.UB = H_kv * g.HB;
@@ -190,7 +194,7 @@ extern "C" int gqa_kv_append_multi(const void *k_new, const void *v_new, void *k
                                    cudaStream_t stream) {
     if (!k_new || !v_new || !k_cache || !v_cache || !seq_lens) return GQA_ERR_NULL;
     if (dtype != GQA_DTYPE_F32 && dtype != GQA_DTYPE_BF16) return GQA_ERR_UNSUPPORTED_DTYPE;
-    if (B <= 0 || Q <= 0 || Q > 64 || H_kv <= 0 || L_max <= 0 ||
+    if (B <= 0 || Q <= 0 || Q > kMaxUnitCols || H_kv <= 0 || L_max <= 0 ||
         static_cast<long long>(B) * H_kv > (1ll << 30))
         return GQA_ERR_SHAPE;
     if (d != 64 && d != 128) return GQA_ERR_UNSUPPORTED_DIM;
@@ -206,7 +210,7 @@ extern "C" int gqa_kv_append_multi(const void *k_new, const void *v_new, void *k
 
 extern "C" size_t gqa_decode_multi_workspace_size(int B, int Q, int H_q, int H_kv, int d,
                                                   gqa_dtype_t dtype) {
-    if (Q < 1 || Q > 64 || check_shape(B, H_q, H_kv, d, 1, dtype) != GQA_OK) return 0;
+    if (Q < 1 || Q > kMaxUnitCols || check_shape(B, H_q, H_kv, d, 1, dtype) != GQA_OK) return 0;
     int dev = 0;
     const int sms = current_sm_count(&dev);
     if (sms <= 0) return 0;
@@ -266,7 +270,7 @@ int decode_impl(const void *q, const void *k_cache, const void *v_cache, const i
     int dev = 0;
     const int sms = current_sm_count(&dev);
     if (sms <= 0) return GQA_ERR_NO_DEVICE;
-    if (Q < 1 || Q > 64) return GQA_ERR_SHAPE;
+    if (Q < 1 || Q > kMaxUnitCols) return GQA_ERR_SHAPE;
     const Geometry g = geometry(B, H_q, H_kv, d, sms, Q);
     if (workspace_bytes < g.bytes) return GQA_ERR_WORKSPACE;
     if (g.slot_floats % 4 != 0 || g.slot_base % 4 != 0) return GQA_ERR_SHAPE;  // 16-byte slot vectors
@@ -455,7 +459,7 @@ extern "C" int gqa_decode_multi(const void *q, const void *k_cache, const void *
                                 int L_max, float scale, gqa_dtype_t dtype, float *out,
                                 void *workspace, size_t workspace_bytes, int32_t *status,
                                 cudaStream_t stream) {
-    if (Q < 1 || Q > 64) return GQA_ERR_SHAPE;
+    if (Q < 1 || Q > kMaxUnitCols) return GQA_ERR_SHAPE;
     return decode_impl(q, k_cache, v_cache, seq_lens, B, H_q, H_kv, d, L_max, 0, scale, dtype,
                        out, workspace, workspace_bytes, status, stream, PagedArgs(), Q);
 }

@@ -66,7 +66,9 @@ struct TcCfg {
     static constexpr int LOG2NHW = NHW >= 16 ? 4 : NHW >= 8 ? 3 : NHW >= 4 ? 2 : NHW >= 2 ? 1 : 0;
 
     struct Small {
-        uint64_t kv_full[8], kv_empty[8];
+        // K and V of a stage land on separate barriers: S = K.Q^T starts as soon as K is in,
+        // while V is still on its way; the stage is released after P.V
+        uint64_t k_full[8], v_full[8], kv_empty[8];
         uint64_t ap_full[8];    // fused append: the copy of a tile that holds the appended row
         uint64_t q_full[2], q_empty[2];
         uint64_t s_full[2], s_empty[2], p_full[2], o_full[2], o_empty[2];
@@ -141,15 +143,17 @@ __device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t bytes) {
 // The ticket warp under a fused append (gqa_kv_append_decode).  Besides the partial pieces'
 // tickets (run_ticket_warp), it owns the appended rows: for every tile that holds a unit's row
 // n - 1, it writes the new K and V rows (k_new, v_new) to the cache for later steps and, once
-// the tile's TMA copy has landed (that copy completes on ap_full instead of kv_full), over the
-// row the copy brought into the ring stage; then it completes the stage's kv_full itself, which
-// releases the tile to the tensor cores and the softmax warps as for any other tile.  The copy
+// the tile's TMA copy has landed (that copy, K and V, completes on ap_full instead of k_full and
+// v_full), over the row the copy brought into the ring stage; then it completes the stage's
+// k_full and v_full itself, which releases the tile to the tensor cores and the softmax warps as
+// for any other tile.  The copy
 // may read the row before or after the cache write; nothing else in the kernel reads it.  An
 // event loop serves whichever of the next row and the next ticket is ready first.  Returns
 // false when a wait ran out.
 template <int D, int NG, int S, int STAGE_BYTES, int TILE_BYTES>
 __device__ bool append_ticket_warp(const DecodeParams &p, const CtaRange &cr, uint8_t *st_base,
-                                   uint64_t *kv_full, uint64_t *ap_full, uint64_t (*pc_full)[2],
+                                   uint64_t *k_full, uint64_t *v_full, uint64_t *ap_full,
+                                   uint64_t (*pc_full)[2],
                                    uint64_t (*tk_done)[2], int (*tk_last)[2], int lane,
                                    const volatile int *abort_flag, uint64_t budget) {
     constexpr int T = 128;
@@ -196,7 +200,7 @@ __device__ bool append_ticket_warp(const DecodeParams &p, const CtaRange &cr, ui
     const int half = lane / CH, c = lane % CH;
     // Per stage, the parity of its next ap_full phase: a stage's patched copies complete in
     // order, and the producer issues the next one only after this warp released the previous
-    // (kv_full -> S.K^T -> P.V -> kv_empty), so the phases never run ahead of this warp.
+    // (k_full, v_full -> S.K^T, P.V -> kv_empty), so the phases never run ahead of this warp.
     uint32_t ap_phase = 0;
     uint64_t idle_since = global_timer_ns();
     uint32_t idle_polls = 0;
@@ -227,7 +231,10 @@ __device__ bool append_ticket_warp(const DecodeParams &p, const CtaRange &cr, ui
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&kv_full[st]);
+                if (lane == 0) {
+                    mbar_arrive(&k_full[st]);
+                    mbar_arrive(&v_full[st]);
+                }
                 next_row();
                 progress = true;
             }
@@ -250,9 +257,13 @@ __device__ bool append_ticket_warp(const DecodeParams &p, const CtaRange &cr, ui
         }
         if (progress) {
             idle_polls = 0;
-        } else if ((++idle_polls & 15u) == 0) {
-            if (idle_polls == 16) idle_since = global_timer_ns();
-            if (*abort_flag || global_timer_ns() - idle_since > budget) return false;
+        } else {
+            // back off between polls: this warp shares its scheduler with a softmax warp
+            __nanosleep(64);
+            if ((++idle_polls & 15u) == 0) {
+                if (idle_polls == 16) idle_since = global_timer_ns();
+                if (*abort_flag || global_timer_ns() - idle_since > budget) return false;
+            }
         }
     }
     return true;
@@ -283,7 +294,8 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(&sm->kv_full[s], 1);
+            mbar_init(&sm->k_full[s], 1);
+            mbar_init(&sm->v_full[s], 1);
             mbar_init(&sm->kv_empty[s], 1);
             mbar_init(&sm->ap_full[s], 1);
         }
@@ -419,12 +431,13 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 uint8_t *kdst = st_base + st * C::STAGE_BYTES;
                 uint8_t *vdst = kdst + C::TILE_BYTES;
-                // A tile that holds a fused append's row lands on ap_full; the ticket warp writes
-                // the row over the copy and then completes kv_full itself.
-                uint64_t *full = &sm->kv_full[st];
+                // K lands on k_full, V on v_full.  A tile that holds a fused append's row lands
+                // whole on ap_full; the ticket warp writes the row over the copy and then
+                // completes k_full and v_full itself.
+                uint64_t *kfull = &sm->k_full[st], *vfull = &sm->v_full[st];
                 ap_mask &= ~(1u << st);
                 if (!PAGED && sg.appended && sg.j0 + sg.len == sg.nt && jj == sg.len - 1) {
-                    full = &sm->ap_full[st];
+                    kfull = vfull = &sm->ap_full[st];
                     ap_mask |= 1u << st;   // the copy now in flight in stage st lands on ap_full
                     ap_par ^= 1u << st;    // with the phase parity before this flip
                 }
@@ -432,7 +445,10 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     // boxes of min(page_size, T) rows, or 8 rows for a partial tile
                     const int boxr = rows == T ? min(p.page_size, T) : 8;
                     const int nbox = rows == T ? T / boxr : (rows + 7) >> 3;
-                    if (lane == 0) mbar_arrive_expect_tx(&sm->kv_full[st], 2 * C::KB * nbox * boxr * 128);
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(&sm->k_full[st], C::KB * nbox * boxr * 128);
+                        mbar_arrive_expect_tx(&sm->v_full[st], C::KB * nbox * boxr * 128);
+                    }
                     __syncwarp();
                     if (lane < nbox) {
                         if (pg < 0 || pg >= p.n_pages) {
@@ -444,27 +460,42 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         const int pr = (row0 + lane * boxr) % p.page_size;
 #pragma unroll
                         for (int kb = 0; kb < C::KB; ++kb) {
-                            tma_load_4d(kdst + kb * T * 128 + lane * boxr * 128, mk, &sm->kv_full[st], kb * 64, sg.kvh, pr, pg, pol);
-                            tma_load_4d(vdst + kb * T * 128 + lane * boxr * 128, mv, &sm->kv_full[st], kb * 64, sg.kvh, pr, pg, pol);
+                            tma_load_4d(kdst + kb * T * 128 + lane * boxr * 128, mk, &sm->k_full[st], kb * 64, sg.kvh, pr, pg, pol);
+                            tma_load_4d(vdst + kb * T * 128 + lane * boxr * 128, mv, &sm->v_full[st], kb * 64, sg.kvh, pr, pg, pol);
                         }
                     }
                 } else if (lane == 0) {
+                    // (one arrival per barrier: on ap_full, K and V together)
                     if (rows == T) {
-                        mbar_arrive_expect_tx(full, C::STAGE_BYTES);
-#pragma unroll
-                        for (int kb = 0; kb < C::KB; ++kb) {
-                            tma_load_4d(kdst + kb * T * 128, &tm_k, full, kb * 64, sg.kvh, row0, sg.b, pol);
-                            tma_load_4d(vdst + kb * T * 128, &tm_v, full, kb * 64, sg.kvh, row0, sg.b, pol);
+                        if (kfull == vfull) {
+                            mbar_arrive_expect_tx(kfull, C::STAGE_BYTES);
+                        } else {
+                            mbar_arrive_expect_tx(kfull, C::TILE_BYTES);
+                            mbar_arrive_expect_tx(vfull, C::TILE_BYTES);
                         }
+#pragma unroll
+                        for (int kb = 0; kb < C::KB; ++kb)
+                            tma_load_4d(kdst + kb * T * 128, &tm_k, kfull, kb * 64, sg.kvh, row0, sg.b, pol);
+#pragma unroll
+                        for (int kb = 0; kb < C::KB; ++kb)
+                            tma_load_4d(vdst + kb * T * 128, &tm_v, vfull, kb * 64, sg.kvh, row0, sg.b, pol);
                     } else {
                         const int nb = (rows + 7) >> 3;  // 8-row boxes: at most 7 rows past n
-                        mbar_arrive_expect_tx(full, 2 * C::KB * nb * 8 * 128);
+                        if (kfull == vfull) {
+                            mbar_arrive_expect_tx(kfull, 2 * C::KB * nb * 8 * 128);
+                        } else {
+                            mbar_arrive_expect_tx(kfull, C::KB * nb * 8 * 128);
+                            mbar_arrive_expect_tx(vfull, C::KB * nb * 8 * 128);
+                        }
                         for (int x = 0; x < nb; ++x) {
 #pragma unroll
-                            for (int kb = 0; kb < C::KB; ++kb) {
-                                tma_load_4d(kdst + kb * T * 128 + x * 1024, &tm_k8, full, kb * 64, sg.kvh, row0 + 8 * x, sg.b, pol);
-                                tma_load_4d(vdst + kb * T * 128 + x * 1024, &tm_v8, full, kb * 64, sg.kvh, row0 + 8 * x, sg.b, pol);
-                            }
+                            for (int kb = 0; kb < C::KB; ++kb)
+                                tma_load_4d(kdst + kb * T * 128 + x * 1024, &tm_k8, kfull, kb * 64, sg.kvh, row0 + 8 * x, sg.b, pol);
+                        }
+                        for (int x = 0; x < nb; ++x) {
+#pragma unroll
+                            for (int kb = 0; kb < C::KB; ++kb)
+                                tma_load_4d(vdst + kb * T * 128 + x * 1024, &tm_v8, vfull, kb * 64, sg.kvh, row0 + 8 * x, sg.b, pol);
                         }
                     }
                 }
@@ -477,20 +508,22 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             // patched tile's copy completes on ap_full, which the ticket warp waits for).
             for (int ii = (i > S ? i - S : 0); ii < i; ++ii) {
                 const int st = ii % S;
-                if (ap_mask & (1u << st))
+                if (ap_mask & (1u << st)) {
                     wait_bounded(&sm->ap_full[st], ((ap_par >> st) & 1u) ^ 1u, nullptr, kDrainNs);
-                else
-                    wait_bounded(&sm->kv_full[st], (ii / S) & 1, nullptr, kDrainNs);
+                } else {
+                    wait_bounded(&sm->k_full[st], (ii / S) & 1, nullptr, kDrainNs);
+                    wait_bounded(&sm->v_full[st], (ii / S) & 1, nullptr, kDrainNs);
+                }
             }
             for (int ss = (sidx > C::QB ? sidx - C::QB : 0); ss < sidx; ++ss)
                 wait_bounded(&sm->q_full[ss % C::QB], (ss / C::QB) & 1, nullptr, kDrainNs);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------------ UMMA issuer
-        // An event loop: a tile's S^T = K.Q^T is issued once its K/V stage has landed and its
-        // S buffer is free; its O^T = V^T.P^T once the softmax warps have written its P.  Each
-        // is issued as soon as it is ready, so releasing a stage never waits for the next
-        // tile's data to arrive.
+        // An event loop: a tile's S^T = K.Q^T is issued once its K tile has landed and its S
+        // buffer is free; its O^T = V^T.P^T once its V tile has landed and the softmax warps
+        // have written its P.  Each is issued as soon as it is ready, so releasing a stage
+        // never waits for the next tile's data to arrive.
         if (lane == 0) {
             // K tile and Q: K-major (rows / heads by d), 8-row groups 1024 B apart.
             // V^T: MN-major (d by rows): the two 64-column blocks T*128 B apart.
@@ -515,7 +548,7 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     if (!q_ready) q_ready = mbar_test_wait(&sm->q_full[qb], (sidx / C::QB) & 1);
                     const int st = qk_t % S;
                     const int j2 = qk_t & 1;
-                    if (q_ready && mbar_test_wait(&sm->kv_full[st], (qk_t / S) & 1) &&
+                    if (q_ready && mbar_test_wait(&sm->k_full[st], (qk_t / S) & 1) &&
                         (qk_t < 2 || mbar_test_wait(&sm->s_empty[j2], ((qk_t >> 1) - 1) & 1))) {
                         tc_fence_after_sync();
                         const uint64_t dk = desc_add(dk0, st * C::STAGE_BYTES);
@@ -542,6 +575,7 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 if (pv_t < qk_t) {
                     const int j2 = pv_t & 1;
                     if (mbar_test_wait(&sm->p_full[j2], (pv_t >> 1) & 1) &&
+                        mbar_test_wait(&sm->v_full[pv_t % S], (pv_t / S) & 1) &&
                         (pv_t < 2 || mbar_test_wait(&sm->o_empty[j2], ((pv_t >> 1) - 1) & 1))) {
                         tc_fence_after_sync();
                         const uint64_t dv = desc_add(dv0, (pv_t % S) * C::STAGE_BYTES);
@@ -577,7 +611,7 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // ------------------------------------------------------------------ ticket warp
         if (!PAGED && p.append) {
             if (!append_ticket_warp<D, C::NWG, S, C::STAGE_BYTES, C::TILE_BYTES>(
-                    p, cr, st_base, sm->kv_full, sm->ap_full, sm->pc_full, sm->tk_done, sm->tk_last, lane,
+                    p, cr, st_base, sm->k_full, sm->v_full, sm->ap_full, sm->pc_full, sm->tk_done, sm->tk_last, lane,
                     abort_flag, budget) &&
                 lane == 0)
                 fail();
@@ -628,7 +662,7 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             for (int jj = 0; jj < sg.len; ++jj, ++i) {
                 const int j2 = i & 1;
                 const int rows = min(T, sg.n - sg.first - (sg.j0 + jj) * T);
-                if (rows < T && !bad && wait_bounded(&sm->kv_full[i % S], (i / S) & 1, abort_flag, budget)) {
+                if (rows < T && !bad && wait_bounded(&sm->v_full[i % S], (i / S) & 1, abort_flag, budget)) {
                     // Rows past n: zero V in shared memory so that 0-weight rows add exactly 0
                     // (stale or unread data there may hold NaN or Inf).
                     uint8_t *vbase = st_base + (i % S) * C::STAGE_BYTES + C::TILE_BYTES;
@@ -897,8 +931,7 @@ static int launch_split_tc_d(const TmaMaps &maps, const DecodeParams &p, int nh,
         case 4: return launch_split_tc_impl<D, 4, PAGED>(maps, p, stream);
         case 8: return launch_split_tc_impl<D, 8, PAGED>(maps, p, stream);
         case 16: return launch_split_tc_impl<D, 16, PAGED>(maps, p, stream);
-        case 32: return launch_split_tc_impl<D, 32, PAGED>(maps, p, stream);
-        default: return launch_split_tc_impl<D, 64, PAGED>(maps, p, stream);
+        default: return launch_split_tc_impl<D, 32, PAGED>(maps, p, stream);  // units have <= 32 columns
     }
 }
 

@@ -78,7 +78,9 @@ struct Tc8Cfg {
     static constexpr int LOG2NHW = NHW >= 16 ? 4 : NHW >= 8 ? 3 : NHW >= 4 ? 2 : NHW >= 2 ? 1 : 0;
 
     struct Small {
-        uint64_t kv_full[8], kv_empty[8];
+        // K and V of a stage land on separate barriers: S = K.Q^T starts as soon as K is in,
+        // while V is still on its way; the stage is released after P.V
+        uint64_t k_full[8], v_full[8], kv_empty[8];
         uint64_t q_full[2], q_empty[2], qf_empty[2];
         uint64_t s_full[2], s_empty[2], p_full[2], o_full[2], o_empty[2];
         uint64_t mma_done;
@@ -194,7 +196,8 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(&sm->kv_full[s], 1);
+            mbar_init(&sm->k_full[s], 1);
+            mbar_init(&sm->v_full[s], 1);
             mbar_init(&sm->kv_empty[s], 1);
         }
         for (int j = 0; j < 2; ++j) {
@@ -408,7 +411,10 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                     boxr = rows == T ? T : 8;
                     nbox = rows == T ? 1 : (rows + 7) >> 3;
                 }
-                if (lane == 0) mbar_arrive_expect_tx(&sm->kv_full[st], 2 * nbox * boxr * ROWB);
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&sm->k_full[st], nbox * boxr * ROWB);
+                    mbar_arrive_expect_tx(&sm->v_full[st], nbox * boxr * ROWB);
+                }
                 __syncwarp();
                 if (lane < nbox) {
                     const CUtensorMap *mk = rows == T ? &tm_k : &tm_k8;
@@ -420,11 +426,11 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                             pg = 0;
                         }
                         const int pr = (row0 + lane * boxr) % p.page_size;
-                        tma_load_4d(kdst + off, mk, &sm->kv_full[st], 0, sg.kvh, pr, pg, pol);
-                        tma_load_4d(vdst + off, mv, &sm->kv_full[st], 0, sg.kvh, pr, pg, pol);
+                        tma_load_4d(kdst + off, mk, &sm->k_full[st], 0, sg.kvh, pr, pg, pol);
+                        tma_load_4d(vdst + off, mv, &sm->v_full[st], 0, sg.kvh, pr, pg, pol);
                     } else {
-                        tma_load_4d(kdst + off, mk, &sm->kv_full[st], 0, sg.kvh, row0 + lane * boxr, sg.b, pol);
-                        tma_load_4d(vdst + off, mv, &sm->kv_full[st], 0, sg.kvh, row0 + lane * boxr, sg.b, pol);
+                        tma_load_4d(kdst + off, mk, &sm->k_full[st], 0, sg.kvh, row0 + lane * boxr, sg.b, pol);
+                        tma_load_4d(vdst + off, mv, &sm->v_full[st], 0, sg.kvh, row0 + lane * boxr, sg.b, pol);
                     }
                 }
                 ++i;
@@ -433,8 +439,10 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         }
         if (lane == 0) {
             if (!ok) fail();
-            for (int ii = (i > S ? i - S : 0); ii < i; ++ii)
-                wait_bounded(&sm->kv_full[ii % S], (ii / S) & 1, nullptr, kDrainNs8);
+            for (int ii = (i > S ? i - S : 0); ii < i; ++ii) {
+                wait_bounded(&sm->k_full[ii % S], (ii / S) & 1, nullptr, kDrainNs8);
+                wait_bounded(&sm->v_full[ii % S], (ii / S) & 1, nullptr, kDrainNs8);
+            }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------------ UMMA issuer
@@ -462,6 +470,7 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                     const int j2 = pv_t & 1;
                     const int ob = pv_t % C::OB;
                     if (mbar_test_wait(&sm->p_full[j2], (pv_t >> 1) & 1) &&
+                        mbar_test_wait(&sm->v_full[pv_t % S], (pv_t / S) & 1) &&
                         (pv_t < C::OB || mbar_test_wait(&sm->o_empty[ob], ((pv_t / C::OB) - 1) & 1))) {
                         tc_fence_after_sync();
                         const uint64_t dv = desc_add8(dv0, (pv_t % S) * C::STAGE_BYTES);
@@ -482,7 +491,7 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                     if (!q_ready) q_ready = mbar_test_wait(&sm->q_full[qb], (sidx / C::QB) & 1);
                     const int st = qk_t % S;
                     const int j2 = qk_t & 1;
-                    if (q_ready && mbar_test_wait(&sm->kv_full[st], (qk_t / S) & 1) &&
+                    if (q_ready && mbar_test_wait(&sm->k_full[st], (qk_t / S) & 1) &&
                         (qk_t < 2 || mbar_test_wait(&sm->s_empty[j2], ((qk_t >> 1) - 1) & 1))) {
                         tc_fence_after_sync();
                         const uint64_t dk = desc_add8(dk0, st * C::STAGE_BYTES);
@@ -616,7 +625,7 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             for (int jj = 0; jj < sg.len; ++jj, ++i) {
                 const int j2 = i & 1;
                 const int rows = min(T, sg.n - sg.first - (sg.j0 + jj) * T);
-                if (rows < T && !bad && wait_bounded(&sm->kv_full[i % S], (i / S) & 1, abort_flag, budget)) {
+                if (rows < T && !bad && wait_bounded(&sm->v_full[i % S], (i / S) & 1, abort_flag, budget)) {
                     // Rows past n: zero V so that 0-weight rows add exactly 0.
                     uint8_t *vbase = st_base + (i % S) * C::STAGE_BYTES + C::TILE_BYTES;
                     constexpr int CPR = ROWB / 16;
@@ -839,8 +848,7 @@ int launch_split_tc8_d(const TmaMaps &maps, const void *q, const DecodeParams &p
         case 4: return launch_split_tc8_impl<D, 4, PAGED>(maps, q, p, stream);
         case 8: return launch_split_tc8_impl<D, 8, PAGED>(maps, q, p, stream);
         case 16: return launch_split_tc8_impl<D, 16, PAGED>(maps, q, p, stream);
-        case 32: return launch_split_tc8_impl<D, 32, PAGED>(maps, q, p, stream);
-        default: return launch_split_tc8_impl<D, 64, PAGED>(maps, q, p, stream);
+        default: return launch_split_tc8_impl<D, 32, PAGED>(maps, q, p, stream);  // units have <= 32 columns
     }
 }
 

@@ -1,7 +1,7 @@
 // Work partition and piece merge shared by the split-KV kernels.
 //
 // The decode work is cut into tiles of T cached rows.  A "unit" is one (sequence b, key/value
-// head j, block of up to 64 query heads of j's group); a unit has ceil(n_b / T) tiles.  Units
+// head j, block of up to 32 query heads of j's group); a unit has ceil(n_b / T) tiles.  Units
 // are ordered b-major, and the tiles of all units form one line of `total` tiles.  The split
 // kernel runs G persistent CTAs and CTA i takes the contiguous tile range
 //     [floor(i * total / G), floor((i + 1) * total / G)),
@@ -29,7 +29,7 @@ struct DecodeParams {
     int r;     // query heads per key/value head
     int Q;     // query tokens per sequence (1, or several for speculative verification)
     int rb;    // query heads per unit and token; a unit's columns are (token j, head h') pairs
-    int RB;    // columns per unit = Q * rb (<= 64), column index j * rb + h'
+    int RB;    // columns per unit = Q * rb (<= 32), column index j * rb + h'
     int HB;    // units per key/value head = ceil(r / rb)
     int q_box_bytes;  // bytes of the q tile of one unit (bf16 path)
     int UB;    // units per sequence = H_kv * HB
@@ -97,13 +97,20 @@ __device__ __forceinline__ int seq_tiles(int n, const DecodeParams &p) {
     return tiles_of(n - first_row(n, p.window), p.T);
 }
 
+// a / b for a >= 0, b > 0: a 32-bit division whenever both fit in 32 bits (the 64-bit one is
+// a long emulated sequence, and the partition arithmetic sits on every CTA's start-up path).
+__device__ __forceinline__ long long udiv(long long a, long long b) {
+    if (((a | b) >> 32) == 0) return static_cast<unsigned>(a) / static_cast<unsigned>(b);
+    return a / b;
+}
+
 __device__ __forceinline__ long long cta_range_begin(long long i, long long total, long long G) {
-    return i * total / G;
+    return udiv(i * total, G);
 }
 
 // The CTA whose range holds tile t (the largest i with begin(i) <= t).
 __device__ __forceinline__ long long cta_of_tile(long long t, long long total, long long G) {
-    return ((t + 1) * G - 1) / total;
+    return udiv((t + 1) * G - 1, total);
 }
 
 __device__ __forceinline__ long long warp_incl_scan(long long v, int lane) {
@@ -239,7 +246,7 @@ struct SegmentWalker {
             offl = cr.offl;
             nl = rows_of(bl, appl);
             ntl = tiles_of(nl - first_row(nl, window), T);
-            kl = static_cast<int>((end - 1 - offl) / ntl);
+            kl = static_cast<int>(udiv(end - 1 - offl, ntl));
             const long long uoffl = offl + static_cast<long long>(kl) * ntl;
             if (uoffl > t) {  // more than one segment: the last one is [uoffl, end)
                 last_first = true;
@@ -282,7 +289,7 @@ struct SegmentWalker {
             nt = tiles_of(n - first_row(n, window), T);
         }
         const long long rel = t - off;
-        const int k = static_cast<int>(rel / nt);
+        const int k = static_cast<int>(udiv(rel, nt));
         const int j0 = static_cast<int>(rel - static_cast<long long>(k) * nt);
         const long long left = end - t;
         const int len = static_cast<int>(left < nt - j0 ? left : nt - j0);

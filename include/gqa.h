@@ -193,7 +193,7 @@ int gqa_decode_window(const void *q, const void *k_cache, const void *v_cache,
  *   t .. t+Q-1, t = seq_lens[b]; then seq_lens[b] = t + Q.  t + Q > L_max (or t < 0) is
  *   refused with GQA_STATUS_APPEND_OVERFLOW.
  * gqa_decode_multi: q [B][Q][H_q][d] -> out [B][Q][H_q][d] (float32); seq_lens[b] >= Q, else
- *   out[b] = 0 and GQA_STATUS_SEQLEN_RANGE.  1 <= Q <= 64.  The workspace is
+ *   out[b] = 0 and GQA_STATUS_SEQLEN_RANGE.  1 <= Q <= 32.  The workspace is
  *   gqa_decode_multi_workspace_size(B, Q, ...) bytes.  Other arguments as gqa_decode.
  */
 int gqa_kv_append_multi(const void *k_new, const void *v_new, void *k_cache, void *v_cache,

@@ -49,7 +49,7 @@ def test_full_size_workloads(oracle, name):
     assert err <= TOL[w.dtype], f"{name}: max abs error {err}"
 
 
-# group sizes 1..128 (128 = two blocks of 64 query heads), both head dims, lengths spanning
+# group sizes 1..128 (64 and 128 = two and four blocks of 32 query heads), both head dims, lengths spanning
 # several 128-row tiles with ragged tails (1, 7, 8, 9, 127, 128, 129, 255, 256, 257, 1000)
 BF16_SHAPES = [
     (3, 8, 8, 128),    # MHA

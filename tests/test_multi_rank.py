@@ -47,7 +47,9 @@ class _StubReplica:
     def time_kernel(self, n, secs):
         return [100.0 + 10 * self.rank] * 5
 
-    def time_steps(self, K, W):
+    def time_steps(self, K, W, barrier=None):
+        if barrier is not None:
+            barrier()
         return K * (1.0 + self.rank)
 
     def time_e2e(self, K, W):
