@@ -292,7 +292,7 @@ int decode_impl(const void *q, const void *k_cache, const void *v_cache, const i
     p.RB = g.RB;
     p.HB = g.HB;
     p.UB = g.UB;
-    p.T = fp8 ? tc8_tile_rows(g.RB) : (dtype == GQA_DTYPE_BF16 ? 128 : 64);
+    p.T = fp8 ? tc8_tile_rows(g.RB) : (dtype == GQA_DTYPE_BF16 ? tc_tile_rows(d, g.RB) : 64);
     p.k_scale = k_scale;
     p.v_scale = v_scale;
     p.k_new = ap.k_new;
@@ -341,7 +341,7 @@ int decode_impl(const void *q, const void *k_cache, const void *v_cache, const i
         // The cache as (d, H_kv, rows, sequences) -- or, paged, (d, H_kv, page_size, n_pages).
         const int rows_dim = pg.block_table ? pg.page_size : L_max;
         const int outer_dim = pg.block_table ? pg.n_pages : B;
-        const int box = pg.block_table ? (pg.page_size < 128 ? pg.page_size : 128) : 128;
+        const int box = pg.block_table ? (pg.page_size < p.T ? pg.page_size : p.T) : p.T;
         (void)rp;
         if (!encode_q_map(&maps.q, q, B, Q, H_q, d, g.rb) ||
             !encode_cache_map(&maps.k, k_cache, outer_dim, H_kv, d, rows_dim, box) ||
@@ -443,8 +443,12 @@ extern "C" int gqa_decode_paged(const void *q, const void *k_pool, const void *v
     if (max_pages <= 0 || n_pages <= 0 || page_size <= 0 || page_size % 8 != 0 ||
         static_cast<long long>(max_pages) * page_size > (1ll << 30))
         return GQA_ERR_SHAPE;
-    // a 128-row tile must lie in one page or cover whole pages
-    if (dtype == GQA_DTYPE_BF16 && 128 % page_size != 0 && page_size % 128 != 0) return GQA_ERR_SHAPE;
+    // a tile (128 rows, or 256 for 64-wide heads of groups up to 8) must lie in one page or
+    // cover whole pages
+    if (dtype == GQA_DTYPE_BF16 && H_kv > 0 && H_q % H_kv == 0) {
+        const int tr = tc_tile_rows(d, H_q / H_kv < 32 ? H_q / H_kv : 32);
+        if (tr % page_size != 0 && page_size % tr != 0) return GQA_ERR_SHAPE;
+    }
     PagedArgs pg;
     pg.block_table = block_table;
     pg.max_pages = max_pages;

@@ -39,7 +39,11 @@ constexpr float kLazyLog2 = 8.0f;
 template <int D, int NH>
 struct TcCfg {
     static constexpr int RP = NH < 16 ? 16 : NH;      // UMMA N of S^T = K.Q^T
-    static constexpr int T = 128;
+    // Rows per softmax thread: 64-wide heads of groups up to 8 columns take 256-row tiles (two
+    // rows a thread, S^T as two 128-lane halves), so that a stage carries 64 KB as at d = 128
+    // and the per-tile chain runs half as often; 128-row tiles otherwise.
+    static constexpr int RPT = (D == 64 && NH <= 8) ? 2 : 1;
+    static constexpr int T = 128 * RPT;
     static constexpr int KB = D / 64;                 // 128-byte column blocks of a row
     static constexpr int TILE_BYTES = T * D * 2;      // one K or V tile
     static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
@@ -51,9 +55,11 @@ struct TcCfg {
     static constexpr int P_ATOMB = T * P_ROWB;
     static constexpr uint32_t P_LAYOUT = P_ROWB == 128 ? 2u : 4u;
     static constexpr int P_BYTES = 2 * RP * T * 2;
-    // TMEM columns: S^T (RP) x2 buffers, then O^T (2*RP: high, low) x2 buffers
-    static constexpr int O_COL = 2 * RP;
-    static constexpr int TMEM_COLS = 6 * RP <= 128 ? 128 : (6 * RP <= 256 ? 256 : 512);
+    // TMEM columns: S^T (RPT halves of RP columns) x2 buffers, then O^T (2*RP: high, low) x2
+    static constexpr int S_BUF = RPT * RP;
+    static constexpr int O_COL = 2 * S_BUF;
+    static constexpr int TMEM_USED = 2 * S_BUF + 4 * RP;
+    static constexpr int TMEM_COLS = TMEM_USED <= 128 ? 128 : (TMEM_USED <= 256 ? 256 : 512);
     static constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, RP, false, false);
     static constexpr uint32_t IDESC_PV = idesc_bf16_f32(D, 2 * RP, true, true);
     // Softmax warpgroups: one for up to 16 heads, else one per 16 heads (heads are
@@ -69,7 +75,8 @@ struct TcCfg {
         // K and V of a stage land on separate barriers: S = K.Q^T starts as soon as K is in,
         // while V is still on its way; the stage is released after P.V
         uint64_t k_full[8], v_full[8], kv_empty[8];
-        uint64_t ap_full[8];    // fused append: the copy of a tile that holds the appended row
+        // fused append: the copies (K, V) of a tile that holds the appended row
+        uint64_t apk_full[8], apv_full[8];
         uint64_t q_full[2], q_empty[2];
         uint64_t s_full[2], s_empty[2], p_full[2], o_full[2], o_empty[2];
         uint64_t mma_done;
@@ -143,20 +150,20 @@ __device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t bytes) {
 // The ticket warp under a fused append (gqa_kv_append_decode).  Besides the partial pieces'
 // tickets (run_ticket_warp), it owns the appended rows: for every tile that holds a unit's row
 // n - 1, it writes the new K and V rows (k_new, v_new) to the cache for later steps and, once
-// the tile's TMA copy has landed (that copy, K and V, completes on ap_full instead of k_full and
-// v_full), over the row the copy brought into the ring stage; then it completes the stage's
-// k_full and v_full itself, which releases the tile to the tensor cores and the softmax warps as
-// for any other tile.  The copy
+// the tile's K copy has landed (it completes on apk_full instead of k_full), over the row the
+// copy brought into the ring stage, and completes the stage's k_full itself, which releases the
+// tile to S = K.Q^T as for any other tile; then the same for V (apv_full, v_full), so the scores
+// never wait for the V half.  The copy
 // may read the row before or after the cache write; nothing else in the kernel reads it.  An
 // event loop serves whichever of the next row and the next ticket is ready first.  Returns
 // false when a wait ran out.
-template <int D, int NG, int S, int STAGE_BYTES, int TILE_BYTES>
+template <int D, int T, int NG, int S, int STAGE_BYTES, int TILE_BYTES>
 __device__ bool append_ticket_warp(const DecodeParams &p, const CtaRange &cr, uint8_t *st_base,
-                                   uint64_t *k_full, uint64_t *v_full, uint64_t *ap_full,
+                                   uint64_t *k_full, uint64_t *v_full, uint64_t *apk_full,
+                                   uint64_t *apv_full,
                                    uint64_t (*pc_full)[2],
                                    uint64_t (*tk_done)[2], int (*tk_last)[2], int lane,
                                    const volatile int *abort_flag, uint64_t budget) {
-    constexpr int T = 128;
     constexpr int CH = D / 8;  // 16-byte chunks of a cached row of one head
     // row cursor: the next tile that holds an appended row
     SegmentWalker wr;
@@ -198,10 +205,12 @@ __device__ bool append_ticket_warp(const DecodeParams &p, const CtaRange &cr, ui
     next_piece();
     const bool mine = lane < 2 * CH;
     const int half = lane / CH, c = lane % CH;
-    // Per stage, the parity of its next ap_full phase: a stage's patched copies complete in
-    // order, and the producer issues the next one only after this warp released the previous
-    // (k_full, v_full -> S.K^T, P.V -> kv_empty), so the phases never run ahead of this warp.
+    // Per stage, the parity of its next apk_full / apv_full phase: a stage's patched copies
+    // complete in order, and the producer issues the next one only after this warp released the
+    // previous (k_full, v_full -> S.K^T, P.V -> kv_empty), so the phases never run ahead of this
+    // warp.  row_half: 0 while the K row is pending, 1 while the V row is.
     uint32_t ap_phase = 0;
+    int row_half = 0;
     uint64_t idle_since = global_timer_ns();
     uint32_t idle_polls = 0;
     while (row_more || tk_more) {
@@ -219,10 +228,10 @@ __device__ bool append_ticket_warp(const DecodeParams &p, const CtaRange &cr, ui
                 row_loaded = true;
             }
             const int st = rt % S;
-            bool landed = lane == 0 ? mbar_test_wait(&ap_full[st], (ap_phase >> st) & 1u) : false;
+            uint64_t *apb = row_half == 0 ? &apk_full[st] : &apv_full[st];
+            bool landed = lane == 0 ? mbar_test_wait(apb, (ap_phase >> st) & 1u) : false;
             if (__shfl_sync(kFullMask, landed, 0)) {
-                ap_phase ^= 1u << st;
-                if (mine) {
+                if (mine && half == row_half) {
                     // row rrow of the stage's K or V tile: 64-column blocks of T rows of 128 bytes,
                     // the 16-byte chunks of a row XOR-swizzled by the row's low three bits
                     uint8_t *base = st_base + st * STAGE_BYTES + half * TILE_BYTES;
@@ -231,11 +240,14 @@ __device__ bool append_ticket_warp(const DecodeParams &p, const CtaRange &cr, ui
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&k_full[st]);
-                    mbar_arrive(&v_full[st]);
+                if (lane == 0) mbar_arrive(row_half == 0 ? &k_full[st] : &v_full[st]);
+                if (row_half == 0) {
+                    row_half = 1;
+                } else {
+                    row_half = 0;
+                    ap_phase ^= 1u << st;
+                    next_row();
                 }
-                next_row();
                 progress = true;
             }
         }
@@ -297,7 +309,8 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mbar_init(&sm->k_full[s], 1);
             mbar_init(&sm->v_full[s], 1);
             mbar_init(&sm->kv_empty[s], 1);
-            mbar_init(&sm->ap_full[s], 1);
+            mbar_init(&sm->apk_full[s], 1);
+            mbar_init(&sm->apv_full[s], 1);
         }
         for (int j = 0; j < 2; ++j) {
             mbar_init(&sm->q_full[j], 1);
@@ -381,7 +394,7 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         Segment sg;
         int i = 0, sidx = 0;
         bool ok = true;
-        uint32_t ap_mask = 0, ap_par = 0;  // fused append: stages whose copy lands on ap_full
+        uint32_t ap_mask = 0, ap_par = 0;  // fused append: stages whose copy lands on apk/apv_full
         [[maybe_unused]] TileCursor ahead;
         [[maybe_unused]] int pg_ring[kPageAhead];
         if constexpr (PAGED) {
@@ -432,13 +445,14 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 uint8_t *kdst = st_base + st * C::STAGE_BYTES;
                 uint8_t *vdst = kdst + C::TILE_BYTES;
                 // K lands on k_full, V on v_full.  A tile that holds a fused append's row lands
-                // whole on ap_full; the ticket warp writes the row over the copy and then
-                // completes k_full and v_full itself.
+                // on apk_full and apv_full instead; the ticket warp writes the row over each
+                // copy and then completes k_full and v_full itself.
                 uint64_t *kfull = &sm->k_full[st], *vfull = &sm->v_full[st];
                 ap_mask &= ~(1u << st);
                 if (!PAGED && sg.appended && sg.j0 + sg.len == sg.nt && jj == sg.len - 1) {
-                    kfull = vfull = &sm->ap_full[st];
-                    ap_mask |= 1u << st;   // the copy now in flight in stage st lands on ap_full
+                    kfull = &sm->apk_full[st];
+                    vfull = &sm->apv_full[st];
+                    ap_mask |= 1u << st;   // the copy now in flight in stage st lands on apk/apv_full
                     ap_par ^= 1u << st;    // with the phase parity before this flip
                 }
                 if constexpr (PAGED) {
@@ -465,14 +479,9 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         }
                     }
                 } else if (lane == 0) {
-                    // (one arrival per barrier: on ap_full, K and V together)
                     if (rows == T) {
-                        if (kfull == vfull) {
-                            mbar_arrive_expect_tx(kfull, C::STAGE_BYTES);
-                        } else {
-                            mbar_arrive_expect_tx(kfull, C::TILE_BYTES);
-                            mbar_arrive_expect_tx(vfull, C::TILE_BYTES);
-                        }
+                        mbar_arrive_expect_tx(kfull, C::TILE_BYTES);
+                        mbar_arrive_expect_tx(vfull, C::TILE_BYTES);
 #pragma unroll
                         for (int kb = 0; kb < C::KB; ++kb)
                             tma_load_4d(kdst + kb * T * 128, &tm_k, kfull, kb * 64, sg.kvh, row0, sg.b, pol);
@@ -481,12 +490,8 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                             tma_load_4d(vdst + kb * T * 128, &tm_v, vfull, kb * 64, sg.kvh, row0, sg.b, pol);
                     } else {
                         const int nb = (rows + 7) >> 3;  // 8-row boxes: at most 7 rows past n
-                        if (kfull == vfull) {
-                            mbar_arrive_expect_tx(kfull, 2 * C::KB * nb * 8 * 128);
-                        } else {
-                            mbar_arrive_expect_tx(kfull, C::KB * nb * 8 * 128);
-                            mbar_arrive_expect_tx(vfull, C::KB * nb * 8 * 128);
-                        }
+                        mbar_arrive_expect_tx(kfull, C::KB * nb * 8 * 128);
+                        mbar_arrive_expect_tx(vfull, C::KB * nb * 8 * 128);
                         for (int x = 0; x < nb; ++x) {
 #pragma unroll
                             for (int kb = 0; kb < C::KB; ++kb)
@@ -505,11 +510,12 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (lane == 0) {
             if (!ok) fail();
             // Drain: no copy may still be writing this CTA's shared memory when it exits (a
-            // patched tile's copy completes on ap_full, which the ticket warp waits for).
+            // patched tile's copies complete on apk_full / apv_full, which the ticket warp waits for).
             for (int ii = (i > S ? i - S : 0); ii < i; ++ii) {
                 const int st = ii % S;
                 if (ap_mask & (1u << st)) {
-                    wait_bounded(&sm->ap_full[st], ((ap_par >> st) & 1u) ^ 1u, nullptr, kDrainNs);
+                    wait_bounded(&sm->apk_full[st], ((ap_par >> st) & 1u) ^ 1u, nullptr, kDrainNs);
+                    wait_bounded(&sm->apv_full[st], ((ap_par >> st) & 1u) ^ 1u, nullptr, kDrainNs);
                 } else {
                     wait_bounded(&sm->k_full[st], (ii / S) & 1, nullptr, kDrainNs);
                     wait_bounded(&sm->v_full[st], (ii / S) & 1, nullptr, kDrainNs);
@@ -554,11 +560,14 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         const uint64_t dk = desc_add(dk0, st * C::STAGE_BYTES);
                         const uint64_t dq = desc_add(dq0, qb * C::Q_BYTES);
 #pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint32_t off_k = (kk >> 2) * T * 128 + (kk & 3) * 32;
-                            const uint32_t off_q = (kk >> 2) * RP * 128 + (kk & 3) * 32;
-                            umma_bf16(tmem + j2 * RP, desc_add(dk, off_k), desc_add(dq, off_q),
-                                      C::IDESC_QK, kk > 0 ? 1u : 0u);
+                        for (int hf = 0; hf < C::RPT; ++hf) {  // 128-row halves of the tile
+#pragma unroll
+                            for (int kk = 0; kk < D / 16; ++kk) {
+                                const uint32_t off_k = (kk >> 2) * T * 128 + hf * 128 * 128 + (kk & 3) * 32;
+                                const uint32_t off_q = (kk >> 2) * RP * 128 + (kk & 3) * 32;
+                                umma_bf16(tmem + j2 * C::S_BUF + hf * RP, desc_add(dk, off_k), desc_add(dq, off_q),
+                                          C::IDESC_QK, kk > 0 ? 1u : 0u);
+                            }
                         }
                         umma_commit(&sm->s_full[j2]);
                         ++qk_t;
@@ -610,8 +619,8 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     } else if (warp == C::TICKET_WARP) {
         // ------------------------------------------------------------------ ticket warp
         if (!PAGED && p.append) {
-            if (!append_ticket_warp<D, C::NWG, S, C::STAGE_BYTES, C::TILE_BYTES>(
-                    p, cr, st_base, sm->k_full, sm->v_full, sm->ap_full, sm->pc_full, sm->tk_done, sm->tk_last, lane,
+            if (!append_ticket_warp<D, T, C::NWG, S, C::STAGE_BYTES, C::TILE_BYTES>(
+                    p, cr, st_base, sm->k_full, sm->v_full, sm->apk_full, sm->apv_full, sm->pc_full, sm->tk_done, sm->tk_last, lane,
                     abort_flag, budget) &&
                 lane == 0)
                 fail();
@@ -676,10 +685,12 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 } else if (rows < T) {
                     bad = true;
                 }
-                uint32_t sr[SCOLS];
+                uint32_t sr[C::RPT][SCOLS];
                 if (!bad && wait_bounded(&sm->s_full[j2], (i >> 1) & 1, abort_flag, budget)) {
                     tc_fence_after_sync();
-                    tmem_ld_cols<SCOLS>(tmem + lane_addr + j2 * RP + hbase, sr);
+#pragma unroll
+                    for (int hf = 0; hf < C::RPT; ++hf)
+                        tmem_ld_cols<SCOLS>(tmem + lane_addr + j2 * C::S_BUF + hf * RP + hbase, sr[hf]);
                     tmem_wait_ld();
                     tc_fence_before_sync();
                     __syncwarp();
@@ -687,18 +698,25 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 } else {
                     bad = true;
 #pragma unroll
-                    for (int h = 0; h < SCOLS; ++h) sr[h] = 0u;
+                    for (int hf = 0; hf < C::RPT; ++hf)
+#pragma unroll
+                        for (int h = 0; h < SCOLS; ++h) sr[hf][h] = 0u;
                 }
 
-                const bool valid = row < rows;
-                // Several query tokens: column j * rb + h' sees rows < n - Q + 1 + j, so a row
-                // `over` rows past n - Q is visible only to columns >= (over + 1) * rb.
-                const int over = sg.first + (sg.j0 + jj) * T + row - (sg.n - p.Q + 1);
-                const int min_col = over >= 0 ? (over + 1) * p.rb : 0;
-                float x[NHW];
+                // This thread's rows of the tile: row, and row + 128 with 256-row tiles.
+                float x[C::RPT][NHW];
 #pragma unroll
-                for (int h = 0; h < NHW; ++h)
-                    x[h] = (valid && hbase + h >= min_col) ? __uint_as_float(sr[h]) * p.scale_log2 : -INFINITY;
+                for (int hf = 0; hf < C::RPT; ++hf) {
+                    const int trow = row + 128 * hf;
+                    const bool valid = trow < rows;
+                    // Several query tokens: column j * rb + h' sees rows < n - Q + 1 + j, so a row
+                    // `over` rows past n - Q is visible only to columns >= (over + 1) * rb.
+                    const int over = sg.first + (sg.j0 + jj) * T + trow - (sg.n - p.Q + 1);
+                    const int min_col = over >= 0 ? (over + 1) * p.rb : 0;
+#pragma unroll
+                    for (int h = 0; h < NHW; ++h)
+                        x[hf][h] = (valid && hbase + h >= min_col) ? __uint_as_float(sr[hf][h]) * p.scale_log2 : -INFINITY;
+                }
                 // Lazy rescaling.  The running maximum m_run only has to keep the exponents in
                 // range, so it is raised -- through an exchange of the warps' tile maxima -- only
                 // when some score of the tile exceeds it by more than kLazyLog2; otherwise every
@@ -706,13 +724,19 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 // either way: P, the running sums and O always share one reference.
                 bool need = false;
 #pragma unroll
-                for (int h = 0; h < NHW; ++h) need |= x[h] > m_run[h] + kLazyLog2;
+                for (int hf = 0; hf < C::RPT; ++hf)
+#pragma unroll
+                    for (int h = 0; h < NHW; ++h) need |= x[hf][h] > m_run[h] + kLazyLog2;
                 if (named_bar_any(bar_id, 128, bad || need)) {
-                    // Per-head maximum over the warp's 32 rows, then over the four warps.
+                    // Per-head maximum over the warp's rows, then over the four warps.
                     {
                         float wm[NHW];
 #pragma unroll
-                        for (int h = 0; h < NHW; ++h) wm[h] = x[h];
+                        for (int h = 0; h < NHW; ++h) {
+                            wm[h] = x[0][h];
+#pragma unroll
+                            for (int hf = 1; hf < C::RPT; ++hf) wm[h] = fmaxf(wm[h], x[hf][h]);
+                        }
                         warp_max_transpose<NHW, C::LOG2NHW>(wm, lane);
                         if (lane < NHW)
                             reinterpret_cast<float *>(&sm->wmax[wg][j2][q4][0])[transpose_head<NHW, C::LOG2NHW>(lane)] = wm[0];
@@ -746,19 +770,21 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     for (int h = 0; h < NHW; ++h) alpha[h] = 1.f;
                 }
 
-                // P = hi + lo in bf16 (~16 significant bits).  This thread's tile row is K row
-                // `row` of the MN-major P^T: high parts at values [0, RP), low parts at
-                // [RP, 2RP), written as 16-byte chunks of 8 heads.
+                // P = hi + lo in bf16 (~16 significant bits).  This thread's tile rows are K rows
+                // of the MN-major P^T: high parts at values [0, RP), low parts at [RP, 2RP),
+                // written as 16-byte chunks of 8 heads.
                 {
-                    uint8_t *prow = p_base + (j2 % C::PB) * C::P_BYTES + row * C::P_ROWB;
-                    const int swz = C::P_ROWB == 128 ? (row & 7) : ((row >> 1) & 3);
                     constexpr int HALF_VALS = C::P_ROWB / 2;  // bf16 values per atom row
 #pragma unroll
                     for (int h = 0; h < NHW; ++h) {
                         // x now holds p; a column with no visible row yet (several query tokens)
                         // keeps p = 0 rather than exp(-inf + inf)
-                        x[h] = x[h] == -INFINITY ? 0.f : ex2_approx(x[h] - m_run[h]);
-                        l[h] = l[h] * alpha[h] + x[h];
+#pragma unroll
+                        for (int hf = 0; hf < C::RPT; ++hf)
+                            x[hf][h] = x[hf][h] == -INFINITY ? 0.f : ex2_approx(x[hf][h] - m_run[h]);
+                        l[h] = l[h] * alpha[h] + x[0][h];
+#pragma unroll
+                        for (int hf = 1; hf < C::RPT; ++hf) l[h] += x[hf][h];
                     }
                     // One P^T buffer: the previous tile's P.V must have read it (its O is folded
                     // below, after this tile's P is handed over).
@@ -766,13 +792,18 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         !wait_bounded(&sm->o_full[(i - 1) & 1], ((i - 1) >> 1) & 1, abort_flag, budget))
                         bad = true;
 #pragma unroll
+                    for (int hf = 0; hf < C::RPT; ++hf) {
+                    const int trow = row + 128 * hf;
+                    uint8_t *prow = p_base + (j2 % C::PB) * C::P_BYTES + trow * C::P_ROWB;
+                    const int swz = C::P_ROWB == 128 ? (trow & 7) : ((trow >> 1) & 3);
+#pragma unroll
                     for (int c8 = 0; c8 < (NHW + 7) / 8; ++c8) {
                         uint32_t hw[4], lw[4];
 #pragma unroll
                         for (int w2 = 0; w2 < 4; ++w2) {
                             const int h = c8 * 8 + 2 * w2;
-                            const float a = h < NHW ? x[h] : 0.f;
-                            const float b = h + 1 < NHW ? x[h + 1] : 0.f;
+                            const float a = h < NHW ? x[hf][h] : 0.f;
+                            const float b = h + 1 < NHW ? x[hf][h + 1] : 0.f;
                             const __nv_bfloat162 hi = __floats2bfloat162_rn(a, b);
                             const __nv_bfloat162 lo = __floats2bfloat162_rn(a - __low2float(hi), b - __high2float(hi));
                             hw[w2] = *reinterpret_cast<const uint32_t *>(&hi);
@@ -783,6 +814,7 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                             make_uint4(hw[0], hw[1], hw[2], hw[3]);
                         *reinterpret_cast<uint4 *>(prow + (el / HALF_VALS) * C::P_ATOMB + ((((el % HALF_VALS) >> 3) ^ swz) << 4)) =
                             make_uint4(lw[0], lw[1], lw[2], lw[3]);
+                    }
                     }
                 }
                 fence_proxy_async_smem();
@@ -940,6 +972,11 @@ int tc_heads_bucket(int heads_per_unit) {
     int nh = 1;
     while (nh < heads_per_unit) nh <<= 1;
     return nh;
+}
+
+// Cached rows per tile of the bf16 kernel for this head dimension and unit width (TcCfg::T).
+int tc_tile_rows(int d, int heads_per_unit) {
+    return (d == 64 && tc_heads_bucket(heads_per_unit) <= 8) ? 256 : 128;
 }
 
 // Rows of the q TMA box: the UMMA N of S^T = K.Q^T.

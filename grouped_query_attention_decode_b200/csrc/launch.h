@@ -20,6 +20,7 @@ struct TmaMaps {
 
 int launch_split_tc(const TmaMaps &maps, const DecodeParams &p, cudaStream_t stream);
 int tc_q_box_rows(int heads_per_unit);
+int tc_tile_rows(int d, int heads_per_unit);
 int launch_split_f32(const DecodeParams &p, const float *q, const float *kc, const float *vc,
                      cudaStream_t stream);
 // FP8 (e4m3) cache: the split kernel (K/V maps of uint8 codes with box rows tc8_tile_rows or

@@ -214,7 +214,8 @@ int gqa_decode_multi(const void *q, const void *k_cache, const void *v_cache,
  * its rows [j*page_size, (j+1)*page_size): row t of sequence b is
  *     k_pool[block_table[b][t / page_size]][t % page_size].
  * Only the entries covering rows < seq_lens[b] (after the append: < seq_lens[b] + 1) are read.
- * page_size must be a multiple of 8 and, for bf16, divide 128 or be a multiple of 128.  A
+ * page_size must be a multiple of 8 and, for bf16, divide the kernel's tile of T rows or be a
+ * multiple of it (T = 256 for d = 64 with groups of up to 8 query heads, else 128).  A
  * sequence's capacity is max_pages * page_size rows (the L_max of the contiguous calls).
  *
  * gqa_kv_append_paged: the append of gqa_kv_append into the pool: row t = seq_lens[b] goes to

@@ -58,6 +58,7 @@ SHAPES = [
     (2, 64, 1, 64),    # r = 64
     (1, 128, 1, 128),  # r = 128: two head blocks share the appended row
     (2, 24, 2, 128),   # r = 12
+    (3, 16, 4, 64),    # r = 4 at d = 64: 256-row tiles
 ]
 
 

@@ -61,6 +61,14 @@ def test_paged_group_sizes(oracle, shape):
     _step(oracle, w, [512, 17, 300][:B], 16)
 
 
+@pytest.mark.parametrize("page_size", [8, 64, 256, 512])
+def test_paged_d64_256_row_tiles(oracle, page_size):
+    # 64-wide heads in groups of up to 8 take 256-row tiles: pages smaller than, equal to and
+    # larger than a tile
+    w = inputs.custom("paged64", B=3, H_q=16, H_kv=2, d=64, L_max=1024, dtype=torch.bfloat16, seed=56)
+    _step(oracle, w, [1024, 257, 40], page_size)
+
+
 @pytest.mark.parametrize("page_size", [8, 24])
 def test_paged_f32(oracle, page_size):
     w = inputs.custom("pagedf", B=3, H_q=8, H_kv=2, d=64, L_max=240, dtype=torch.float32, seed=53)
@@ -94,7 +102,7 @@ def test_paged_bad_page_is_reported(oracle):
 def test_paged_rejects_unsupported_page_size():
     w = inputs.custom("pagedrej", B=1, H_q=8, H_kv=2, d=64, L_max=96, dtype=torch.bfloat16, seed=55)
     x = inputs.make_inputs(w, lengths=[96])
-    pg = inputs.make_paged(x, 24)  # 24 neither divides 128 nor is a multiple of it
+    pg = inputs.make_paged(x, 24)  # 24 neither divides the 256-row tile nor is a multiple of it
     with pytest.raises(gqa.GQAError):
         gqa.decode_paged(x["q"].cuda(), pg["k_pool"].cuda(), pg["v_pool"].cuda(),
                          pg["block_table"].cuda(), x["lengths"].cuda(), x["scale"])

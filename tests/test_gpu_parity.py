@@ -61,6 +61,7 @@ BF16_SHAPES = [
     (1, 128, 1, 128),  # r = 128: two head blocks
     (2, 96, 2, 64),    # r = 48: padded to 64
     (2, 24, 2, 128),   # r = 12: padded to 16
+    (3, 16, 4, 64),    # r = 4 at d = 64: 256-row tiles
 ]
 
 
