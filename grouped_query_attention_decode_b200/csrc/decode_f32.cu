@@ -93,7 +93,7 @@ split_f32_kernel(const float *__restrict__ q, const float *__restrict__ kc,
         for (int k = 0; k < ACC; ++k) acc[k] = 0.f;
         __syncthreads();
         for (int jj = 0; jj < sg.len; ++jj) {
-            const int row0 = sg.first + (sg.j0 + jj) * T;
+            const int row0 = sg.first + sg.tile(jj) * T;
             const int rows = min(T, sg.n - row0);
             for (int idx = tid; idx < rows * (D / 4); idx += 256) {
                 const int t = idx / (D / 4);

@@ -180,7 +180,7 @@ __device__ bool append_ticket_warp(const DecodeParams &p, const CtaRange &cr, ui
             const int first = tile_r;
             tile_r += sr.len;
             if (sr.appended && sr.j0 + sr.len == sr.nt) {
-                rt = first + sr.len - 1;
+                rt = first;  // the piece computes the unit's last tile first
                 rrow = (sr.n - 1) - (sr.first + (sr.nt - 1) * T);
                 row_more = true;
                 return;
@@ -425,7 +425,7 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             ++sidx;
             for (int jj = 0; jj < sg.len; ++jj) {
                 const int st = i % S;
-                const int row0 = sg.first + (sg.j0 + jj) * T;
+                const int row0 = sg.first + sg.tile(jj) * T;
                 const int rows = min(T, sg.n - row0);
                 [[maybe_unused]] int pg = 0;
                 if constexpr (PAGED) {
@@ -449,7 +449,7 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 // copy and then completes k_full and v_full itself.
                 uint64_t *kfull = &sm->k_full[st], *vfull = &sm->v_full[st];
                 ap_mask &= ~(1u << st);
-                if (!PAGED && sg.appended && sg.j0 + sg.len == sg.nt && jj == sg.len - 1) {
+                if (!PAGED && sg.appended && sg.last_tile(jj)) {
                     kfull = &sm->apk_full[st];
                     vfull = &sm->apv_full[st];
                     ap_mask |= 1u << st;   // the copy now in flight in stage st lands on apk/apv_full
@@ -670,7 +670,7 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             bool bad = false;
             for (int jj = 0; jj < sg.len; ++jj, ++i) {
                 const int j2 = i & 1;
-                const int rows = min(T, sg.n - sg.first - (sg.j0 + jj) * T);
+                const int rows = min(T, sg.n - sg.first - sg.tile(jj) * T);
                 if (rows < T && !bad && wait_bounded(&sm->v_full[i % S], (i / S) & 1, abort_flag, budget)) {
                     // Rows past n: zero V in shared memory so that 0-weight rows add exactly 0
                     // (stale or unread data there may hold NaN or Inf).
@@ -711,7 +711,7 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     const bool valid = trow < rows;
                     // Several query tokens: column j * rb + h' sees rows < n - Q + 1 + j, so a row
                     // `over` rows past n - Q is visible only to columns >= (over + 1) * rb.
-                    const int over = sg.first + (sg.j0 + jj) * T + trow - (sg.n - p.Q + 1);
+                    const int over = sg.first + sg.tile(jj) * T + trow - (sg.n - p.Q + 1);
                     const int min_col = over >= 0 ? (over + 1) * p.rb : 0;
 #pragma unroll
                     for (int h = 0; h < NHW; ++h)

@@ -378,7 +378,7 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             }
             for (int jj = 0; jj < sg.len; ++jj) {
                 const int st = i % S;
-                const int row0 = sg.first + (sg.j0 + jj) * T;
+                const int row0 = sg.first + sg.tile(jj) * T;
                 const int rows = min(T, sg.n - row0);
                 [[maybe_unused]] int pg = 0;
                 if constexpr (PAGED) {
@@ -624,7 +624,7 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             ++sidx;
             for (int jj = 0; jj < sg.len; ++jj, ++i) {
                 const int j2 = i & 1;
-                const int rows = min(T, sg.n - sg.first - (sg.j0 + jj) * T);
+                const int rows = min(T, sg.n - sg.first - sg.tile(jj) * T);
                 if (rows < T && !bad && wait_bounded(&sm->v_full[i % S], (i / S) & 1, abort_flag, budget)) {
                     // Rows past n: zero V so that 0-weight rows add exactly 0.
                     uint8_t *vbase = st_base + (i % S) * C::STAGE_BYTES + C::TILE_BYTES;
@@ -654,7 +654,7 @@ split_tc8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 bool need = false;
                 {
                     const bool valid = trow < rows;
-                    const int over = sg.first + (sg.j0 + jj) * T + trow - (sg.n - p.Q + 1);
+                    const int over = sg.first + sg.tile(jj) * T + trow - (sg.n - p.Q + 1);
                     const int min_col = over >= 0 ? (over + 1) * p.rb : 0;
 #pragma unroll
                     for (int h = 0; h < NHW; ++h) {

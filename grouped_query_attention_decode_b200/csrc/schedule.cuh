@@ -198,6 +198,20 @@ struct Segment {
     bool appended;   // a fused append writes row n - 1 of the sequence
     int nt;          // tiles of the unit
     long long uoff;  // line position of the unit's first tile
+
+    // Tile (within the unit) that the piece computes jj-th.  A piece that ends the unit takes
+    // the unit's last tile first: that tile is the one a fused append patches and the one that
+    // is cut short when the length is not a multiple of the tile, and its extra latency then
+    // hides behind the loads of the tiles after it instead of ending the CTA's work.  Online
+    // softmax does not depend on the order; every kernel and the page cursor use this one map.
+    __device__ __forceinline__ int tile(int jj) const {
+        if (j0 + len == nt && len > 1) return jj == 0 ? nt - 1 : j0 + jj - 1;
+        return j0 + jj;
+    }
+    // The piece's jj-th tile is the unit's last one.
+    __device__ __forceinline__ bool last_tile(int jj) const {
+        return j0 + len == nt && (len > 1 ? jj == 0 : true);
+    }
 };
 
 // Walks the segments of one CTA range: its last segment first (when the range has more than
@@ -577,7 +591,7 @@ struct TileCursor {
     // block-table index stays below max_pages.
     __device__ int page_of_box(const DecodeParams &p, int T, int box) const {
         if (!live) return 0;
-        const int row0 = sg.first + (sg.j0 + jj) * T;
+        const int row0 = sg.first + sg.tile(jj) * T;
         const int rows = min(T, sg.n - row0);
         const int boxr = rows == T ? min(p.page_size, T) : 8;
         const int nbox = rows == T ? T / boxr : (rows + 7) >> 3;

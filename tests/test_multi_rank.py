@@ -53,7 +53,7 @@ class _StubReplica:
         return K * (1.0 + self.rank)
 
     def time_e2e(self, K, W):
-        return {"ms_per_step": 2.0 + self.rank, "api_only_ms_per_step": 1.5,
+        return {"ms_per_step": 2.0 + self.rank, "serial_ms_per_step": 2.5, "api_only_ms_per_step": 1.5,
                 "copies_only_ms_per_step": 0.1, "h2d": 10, "d2h": 20}
 
     def read_stream(self):
