@@ -492,12 +492,13 @@ class Replica:
         return e0.elapsed_time(e1)
 
     def time_kernel(self, min_launches: int, min_seconds: float) -> list[float]:
-        """The split-KV kernel alone: a graph of kg back-to-back decode launches (consecutive
-        launches overlap only as programmatic dependent launch allows), replayed until at least
-        min_launches launches and min_seconds; CUDA events around every replay.  Returns the
-        average µs per launch of each replay."""
+        """The split-KV kernel alone: a graph of kg back-to-back launches of it -- the fused
+        append + decode launch when that is the whole step, else the decode launch (consecutive
+        launches overlap only as programmatic dependent launch allows) -- replayed until at
+        least min_launches launches and min_seconds; CUDA events around every replay.  Returns
+        the average µs per launch of each replay."""
         kg = self.n_copies * max(1, -(-100 // self.n_copies))
-        g, keep = self._capture(kg, decode_only=True)
+        g, keep = self._capture(kg, decode_only=not self.fused)
         for _ in range(3):
             g.replay()
         torch.cuda.synchronize()

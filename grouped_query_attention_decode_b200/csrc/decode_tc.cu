@@ -20,7 +20,9 @@
 //   warp 1       UMMA issuer (one elected thread, event loop)
 //   warps 2..    NWG softmax / accumulation / epilogue warpgroups of 128 threads, each owning
 //                a slice of the group's query heads (one warpgroup up to 16 heads)
-//   last warp    ticket warp: takes the tickets of the pieces cut from units (schedule.cuh)
+//   last warp    ticket warp: takes the tickets of the pieces cut from units (schedule.cuh);
+//                under a fused append it also writes the appended rows into the cache and over
+//                the copies of the tiles that hold them
 // Every wait is bounded; on a timeout the CTA drains its in-flight copies and UMMAs, frees
 // its tensor memory, sets GQA_STATUS_WAIT_TIMEOUT and returns.
 #include <cstdint>
@@ -150,134 +152,96 @@ __device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t bytes) {
 // The ticket warp under a fused append (gqa_kv_append_decode).  Besides the partial pieces'
 // tickets (run_ticket_warp), it owns the appended rows: for every tile that holds a unit's row
 // n - 1, it writes the new K and V rows (k_new, v_new) to the cache for later steps and, once
-// the tile's K copy has landed (it completes on apk_full instead of k_full), over the row the
-// copy brought into the ring stage, and completes the stage's k_full itself, which releases the
-// tile to S = K.Q^T as for any other tile; then the same for V (apv_full, v_full), so the scores
-// never wait for the V half.  The copy
-// may read the row before or after the cache write; nothing else in the kernel reads it.  An
-// event loop serves whichever of the next row and the next ticket is ready first.  Returns
-// false when a wait ran out.
+// the tile's K copy has landed (it completes on apk_full instead of k_full), writes the K row
+// over the row the copy brought into the ring stage and completes the stage's k_full itself,
+// which releases the tile to S = K.Q^T as for any other tile; then the same for V (apv_full,
+// v_full), so the scores never wait for the V half.  The copy may read the row before or after
+// the cache write; nothing else in the kernel reads it.
+//
+// Both kinds of event come in the CTA's walk order, and every wait blocks (a blocking mbarrier
+// wait wakes as soon as its phase completes; an earlier version polled both kinds from one
+// loop with a back-off and took the tickets late).  A piece that ends its unit computes the
+// unit's last tile -- the patched one -- first, so segment s's patch is due while segment s - 1
+// is still being computed: the ticket of a partial segment is therefore taken after the next
+// segment's patch, which keeps the patch ahead of the scores that wait for it.  No ticket is
+// urgent before the CTA's last piece, whose ticket follows no patch.  Returns false when a
+// wait ran out.
 template <int D, int T, int NG, int S, int STAGE_BYTES, int TILE_BYTES>
 __device__ bool append_ticket_warp(const DecodeParams &p, const CtaRange &cr, uint8_t *st_base,
                                    uint64_t *k_full, uint64_t *v_full, uint64_t *apk_full,
-                                   uint64_t *apv_full,
-                                   uint64_t (*pc_full)[2],
+                                   uint64_t *apv_full, uint64_t (*pc_full)[2],
                                    uint64_t (*tk_done)[2], int (*tk_last)[2], int lane,
                                    const volatile int *abort_flag, uint64_t budget) {
     constexpr int CH = D / 8;  // 16-byte chunks of a cached row of one head
-    // row cursor: the next tile that holds an appended row
-    SegmentWalker wr;
-    wr.init(p, cr);
-    Segment sr;
-    int tile_r = 0;  // walk index of the next segment's first tile
-    bool row_more = false, row_loaded = false;
-    int rt = 0, rrow = 0;  // walk index of the tile, the row within it
-    uint4 chunk = make_uint4(0, 0, 0, 0);
-    auto next_row = [&]() {
-        row_more = false;
-        row_loaded = false;
-        while (wr.next(sr)) {
-            const int first = tile_r;
-            tile_r += sr.len;
-            if (sr.appended && sr.j0 + sr.len == sr.nt) {
-                rt = first;  // the piece computes the unit's last tile first
-                rrow = (sr.n - 1) - (sr.first + (sr.nt - 1) * T);
-                row_more = true;
-                return;
-            }
-        }
-    };
-    next_row();
-    // ticket cursor: the CTA's partial pieces (at most two), group by group
-    SegmentWalker wt;
-    wt.init(p, cr);
-    Segment stk;
-    int k = 0, g = 0;
-    bool tk_more = false;
-    auto next_piece = [&]() {
-        tk_more = false;
-        while (k < 2 && wt.next(stk))
-            if (!stk.whole) {
-                tk_more = true;
-                return;
-            }
-    };
-    next_piece();
     const bool mine = lane < 2 * CH;
     const int half = lane / CH, c = lane % CH;
+    SegmentWalker w;
+    w.init(p, cr);
+    Segment sg, pend;
+    bool has_pend = false;
+    int tile_r = 0;  // walk index of the next segment's first tile
+    int k = 0;       // partial pieces seen (a CTA has at most two)
     // Per stage, the parity of its next apk_full / apv_full phase: a stage's patched copies
     // complete in order, and the producer issues the next one only after this warp released the
     // previous (k_full, v_full -> S.K^T, P.V -> kv_empty), so the phases never run ahead of this
-    // warp.  row_half: 0 while the K row is pending, 1 while the V row is.
+    // warp.
     uint32_t ap_phase = 0;
-    int row_half = 0;
-    uint64_t idle_since = global_timer_ns();
-    uint32_t idle_polls = 0;
-    while (row_more || tk_more) {
-        bool progress = false;
-        if (row_more) {
-            if (!row_loaded) {
-                // the new row: one 16-byte chunk of K (lanes < CH) or V (the next CH lanes) per
-                // lane, written to the cache at once
-                if (mine) {
-                    const long long src = (static_cast<long long>(sr.b) * p.H_kv + sr.kvh) * CH + c;
-                    chunk = __ldg(static_cast<const uint4 *>(half ? p.v_new : p.k_new) + src);
-                    const long long dst = ((static_cast<long long>(sr.b) * p.L_max + (sr.n - 1)) * p.H_kv + sr.kvh) * CH + c;
-                    static_cast<uint4 *>(half ? p.v_cache : p.k_cache)[dst] = chunk;
-                }
-                row_loaded = true;
+    auto take = [&](const Segment &ps, int kk) {
+        for (int g = 0; g < NG; ++g) {
+            const bool got = wait_bounded(&pc_full[g][kk], 0, abort_flag, budget);
+            if (!__all_sync(kFullMask, got)) return false;
+            if (lane == 0) {
+                int c0, c1;
+                tk_last[g][kk] = take_ticket(p, ps.unit, g) == unit_pieces(ps.uoff, ps.nt, cr.total, p.G, c0, c1) - 1;
+                mbar_arrive(&tk_done[g][kk]);
             }
-            const int st = rt % S;
-            uint64_t *apb = row_half == 0 ? &apk_full[st] : &apv_full[st];
-            bool landed = lane == 0 ? mbar_test_wait(apb, (ap_phase >> st) & 1u) : false;
-            if (__shfl_sync(kFullMask, landed, 0)) {
-                if (mine && half == row_half) {
-                    // row rrow of the stage's K or V tile: 64-column blocks of T rows of 128 bytes,
-                    // the 16-byte chunks of a row XOR-swizzled by the row's low three bits
-                    uint8_t *base = st_base + st * STAGE_BYTES + half * TILE_BYTES;
+        }
+        return true;
+    };
+    while (w.next(sg)) {
+        const int first = tile_r;
+        tile_r += sg.len;
+        if (sg.appended && sg.j0 + sg.len == sg.nt) {
+            // the piece computes the unit's last tile first: walk index `first`
+            const int st = first % S;
+            const int rrow = (sg.n - 1) - (sg.first + (sg.nt - 1) * T);
+            // the new row: one 16-byte chunk of K (lanes < CH) or V (the next CH lanes) per
+            // lane, written to the cache at once
+            uint4 chunk = make_uint4(0, 0, 0, 0);
+            if (mine) {
+                const long long src = (static_cast<long long>(sg.b) * p.H_kv + sg.kvh) * CH + c;
+                chunk = __ldg(static_cast<const uint4 *>(half ? p.v_new : p.k_new) + src);
+                const long long dst = ((static_cast<long long>(sg.b) * p.L_max + (sg.n - 1)) * p.H_kv + sg.kvh) * CH + c;
+                static_cast<uint4 *>(half ? p.v_cache : p.k_cache)[dst] = chunk;
+            }
+            const uint32_t par = (ap_phase >> st) & 1u;
+            for (int hv = 0; hv < 2; ++hv) {
+                const bool landed = wait_bounded(hv == 0 ? &apk_full[st] : &apv_full[st], par, abort_flag, budget);
+                if (!__all_sync(kFullMask, landed)) return false;
+                if (mine && half == hv) {
+                    // row rrow of the stage's K or V tile: 64-column blocks of T rows of 128
+                    // bytes, the 16-byte chunks of a row XOR-swizzled by the row's low three bits
+                    uint8_t *base = st_base + st * STAGE_BYTES + hv * TILE_BYTES;
                     const int kb = c >> 3, cc = c & 7;
                     *reinterpret_cast<uint4 *>(base + kb * T * 128 + rrow * 128 + ((cc ^ (rrow & 7)) << 4)) = chunk;
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(row_half == 0 ? &k_full[st] : &v_full[st]);
-                if (row_half == 0) {
-                    row_half = 1;
-                } else {
-                    row_half = 0;
-                    ap_phase ^= 1u << st;
-                    next_row();
-                }
-                progress = true;
+                if (lane == 0) mbar_arrive(hv == 0 ? &k_full[st] : &v_full[st]);
             }
+            ap_phase ^= 1u << st;
         }
-        if (tk_more) {
-            bool done = lane == 0 ? mbar_test_wait(&pc_full[g][k], 0) : false;
-            if (__shfl_sync(kFullMask, done, 0)) {
-                if (lane == 0) {
-                    int c0, c1;
-                    tk_last[g][k] = take_ticket(p, stk.unit, g) == unit_pieces(stk.uoff, stk.nt, cr.total, p.G, c0, c1) - 1;
-                    mbar_arrive(&tk_done[g][k]);
-                }
-                if (++g == NG) {
-                    g = 0;
-                    ++k;
-                    next_piece();
-                }
-                progress = true;
-            }
+        if (has_pend) {
+            if (!take(pend, k - 1)) return false;
+            has_pend = false;
         }
-        if (progress) {
-            idle_polls = 0;
-        } else {
-            // back off between polls: this warp shares its scheduler with a softmax warp
-            __nanosleep(64);
-            if ((++idle_polls & 15u) == 0) {
-                if (idle_polls == 16) idle_since = global_timer_ns();
-                if (*abort_flag || global_timer_ns() - idle_since > budget) return false;
-            }
+        if (!sg.whole && k < 2) {
+            pend = sg;
+            has_pend = true;
+            ++k;
         }
     }
+    if (has_pend && !take(pend, k - 1)) return false;
     return true;
 }
 
@@ -620,8 +584,8 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // ------------------------------------------------------------------ ticket warp
         if (!PAGED && p.append) {
             if (!append_ticket_warp<D, T, C::NWG, S, C::STAGE_BYTES, C::TILE_BYTES>(
-                    p, cr, st_base, sm->k_full, sm->v_full, sm->apk_full, sm->apv_full, sm->pc_full, sm->tk_done, sm->tk_last, lane,
-                    abort_flag, budget) &&
+                    p, cr, st_base, sm->k_full, sm->v_full, sm->apk_full, sm->apv_full, sm->pc_full, sm->tk_done,
+                    sm->tk_last, lane, abort_flag, budget) &&
                 lane == 0)
                 fail();
         } else {
