@@ -8,7 +8,10 @@
 //
 //   S^T[128 rows x RP heads] = K_tile[128 x d] . Q^T            (UMMA, M=128, N=RP, K=d)
 //   softmax over the 128 rows, online across tiles, in fp32      (4 warps, one row per thread)
-//   O^T[d x 2RP] = V_tile^T[d x 128] . [P_hi | P_lo]^T           (UMMA, M=d, N=2RP, K=128)
+//   O^T[d x PN] = V_tile^T[d x 128] . [P_hi | P_lo]^T            (UMMA, M=d, N=PN, K=128)
+//
+// (tiles of 256 rows at d = 64 for units of up to 8 columns: two S MMAs, two rows per thread,
+// K = 256 for the second product; PN = 2*RP, or 16 for units of up to 8 columns)
 //
 // and the O^T tiles are accumulated with the online-softmax rescale in registers (thread =
 // one of the d output columns).  P enters the second product as two bf16 parts (high, and the
@@ -50,20 +53,26 @@ struct TcCfg {
     static constexpr int TILE_BYTES = T * D * 2;      // one K or V tile
     static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
     static constexpr int Q_BYTES = RP * D * 2;
-    // P^T in bf16, MN-major: tile row r (the K index) holds 2*RP values, the high parts of
-    // heads 0..RP-1 then their low parts.  Rows are 64 bytes (RP = 16, 64-byte swizzle) or
-    // 128 bytes (RP >= 32, 128-byte swizzle); 2*RP > 64 values take two 128-byte atoms.
-    static constexpr int P_ROWB = 4 * RP >= 128 ? 128 : 4 * RP;
+    // P^T in bf16, MN-major: tile row r (the K index) holds PN = 2*LO values, the high parts
+    // of the heads at [0, LO) and their low parts at [LO, 2*LO).  LO = RP, except for units of
+    // up to 8 columns, where one 16-byte chunk holds the 8 high parts and the next the 8 low
+    // parts (LO = 8): P is then half the size, so that two P buffers fit beside a three-stage
+    // ring of 64 KB stages.  Rows are 32 bytes (32-byte swizzle), 64 bytes (RP = 16, 64-byte
+    // swizzle) or 128 bytes (RP >= 32, 128-byte swizzle); PN > 64 values take two 128-byte atoms.
+    static constexpr int LO = NH <= 8 ? 8 : RP;
+    static constexpr int PN = 2 * LO;                 // UMMA N of O^T = V^T.P^T
+    static constexpr int P_ROWB = 2 * PN >= 128 ? 128 : 2 * PN;
     static constexpr int P_ATOMB = T * P_ROWB;
-    static constexpr uint32_t P_LAYOUT = P_ROWB == 128 ? 2u : 4u;
-    static constexpr int P_BYTES = 2 * RP * T * 2;
-    // TMEM columns: S^T (RPT halves of RP columns) x2 buffers, then O^T (2*RP: high, low) x2
+    static constexpr uint32_t P_LAYOUT = P_ROWB == 128 ? 2u : (P_ROWB == 64 ? 4u : 6u);
+    static constexpr int P_BYTES = PN * T * 2;
+    // TMEM columns: S^T (RPT halves of RP columns) x2 buffers, then O^T (PN: high, low) x2
     static constexpr int S_BUF = RPT * RP;
     static constexpr int O_COL = 2 * S_BUF;
-    static constexpr int TMEM_USED = 2 * S_BUF + 4 * RP;
+    static constexpr int OB = PN;                     // columns of one O^T buffer
+    static constexpr int TMEM_USED = 2 * S_BUF + 2 * OB;
     static constexpr int TMEM_COLS = TMEM_USED <= 128 ? 128 : (TMEM_USED <= 256 ? 256 : 512);
     static constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, RP, false, false);
-    static constexpr uint32_t IDESC_PV = idesc_bf16_f32(D, 2 * RP, true, true);
+    static constexpr uint32_t IDESC_PV = idesc_bf16_f32(D, PN, true, true);
     // Softmax warpgroups: one for up to 16 heads, else one per 16 heads (heads are
     // independent, so the groups split them and never exchange data).
     static constexpr int NWG = NH >= 32 ? NH / 16 : 1;
@@ -497,7 +506,7 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (lane == 0) {
             // K tile and Q: K-major (rows / heads by d), 8-row groups 1024 B apart.
             // V^T: MN-major (d by rows): the two 64-column blocks T*128 B apart.
-            // P^T: MN-major (2*RP values per tile row), 8-row groups 8*P_ROWB apart.
+            // P^T: MN-major (PN values per tile row), 8-row groups 8*P_ROWB apart.
             const uint64_t dk0 = sdesc_sw128(smem_u32(st_base), 16, 1024);
             const uint64_t dv0 = sdesc_sw128(smem_u32(st_base + C::TILE_BYTES), T * 128, 1024);
             const uint64_t dq0 = sdesc_sw128(smem_u32(q_base), 16, 1024);
@@ -557,7 +566,7 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         // N = 2*RP product.
 #pragma unroll
                         for (int kk = 0; kk < T / 16; ++kk) {
-                            umma_bf16(tmem + C::O_COL + j2 * C::O_COL, desc_add(dv, kk * 2048),
+                            umma_bf16(tmem + C::O_COL + j2 * C::OB, desc_add(dv, kk * 2048),
                                       desc_add(dp, kk * 16 * C::P_ROWB), C::IDESC_PV, kk > 0 ? 1u : 0u);
                         }
                         umma_commit(&sm->o_full[j2]);
@@ -759,7 +768,7 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     for (int hf = 0; hf < C::RPT; ++hf) {
                     const int trow = row + 128 * hf;
                     uint8_t *prow = p_base + (j2 % C::PB) * C::P_BYTES + trow * C::P_ROWB;
-                    const int swz = C::P_ROWB == 128 ? (trow & 7) : ((trow >> 1) & 3);
+                    const int swz = C::P_ROWB == 128 ? (trow & 7) : (C::P_ROWB == 64 ? ((trow >> 1) & 3) : ((trow >> 2) & 1));
 #pragma unroll
                     for (int c8 = 0; c8 < (NHW + 7) / 8; ++c8) {
                         uint32_t hw[4], lw[4];
@@ -773,7 +782,7 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                             hw[w2] = *reinterpret_cast<const uint32_t *>(&hi);
                             lw[w2] = *reinterpret_cast<const uint32_t *>(&lo);
                         }
-                        const int eh = hbase + c8 * 8, el = RP + hbase + c8 * 8;
+                        const int eh = hbase + c8 * 8, el = C::LO + hbase + c8 * 8;
                         *reinterpret_cast<uint4 *>(prow + (eh / HALF_VALS) * C::P_ATOMB + ((((eh % HALF_VALS) >> 3) ^ swz) << 4)) =
                             make_uint4(hw[0], hw[1], hw[2], hw[3]);
                         *reinterpret_cast<uint4 *>(prow + (el / HALF_VALS) * C::P_ATOMB + ((((el % HALF_VALS) >> 3) ^ swz) << 4)) =
@@ -794,17 +803,26 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         continue;
                     }
                     tc_fence_after_sync();
-                    const uint32_t obase = tmem + lane_addr + C::O_COL + jt * C::O_COL + hbase;
-#pragma unroll
-                    for (int c = 0; c < NHW; c += 16) {
-                        uint32_t hi[16], lo[16];
-                        tmem_ld16(obase + c, hi);
-                        tmem_ld16(obase + RP + c, lo);
+                    const uint32_t obase = tmem + lane_addr + C::O_COL + jt * C::OB + hbase;
+                    if constexpr (C::LO == 8) {
+                        uint32_t v[16];  // high parts in columns 0..7, low parts in 8..15
+                        tmem_ld16(obase, v);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int e = 0; e < 16; ++e)
-                            if (c + e < NHW)
-                                O[c + e] = (O[c + e] + (__uint_as_float(hi[e]) + __uint_as_float(lo[e]))) * alpha[c + e];
+                        for (int e = 0; e < NHW; ++e)
+                            O[e] = (O[e] + (__uint_as_float(v[e]) + __uint_as_float(v[8 + e]))) * alpha[e];
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < NHW; c += 16) {
+                            uint32_t hi[16], lo[16];
+                            tmem_ld16(obase + c, hi);
+                            tmem_ld16(obase + C::LO + c, lo);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int e = 0; e < 16; ++e)
+                                if (c + e < NHW)
+                                    O[c + e] = (O[c + e] + (__uint_as_float(hi[e]) + __uint_as_float(lo[e]))) * alpha[c + e];
+                        }
                     }
                     tc_fence_before_sync();
                     __syncwarp();
@@ -816,16 +834,24 @@ split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 // Last tile of the piece: its O is already relative to the final max.
                 const int jt = (i - 1) & 1;
                 tc_fence_after_sync();
-                const uint32_t obase = tmem + lane_addr + C::O_COL + jt * C::O_COL + hbase;
-#pragma unroll
-                for (int c = 0; c < NHW; c += 16) {
-                    uint32_t hi[16], lo[16];
-                    tmem_ld16(obase + c, hi);
-                    tmem_ld16(obase + RP + c, lo);
+                const uint32_t obase = tmem + lane_addr + C::O_COL + jt * C::OB + hbase;
+                if constexpr (C::LO == 8) {
+                    uint32_t v[16];  // high parts in columns 0..7, low parts in 8..15
+                    tmem_ld16(obase, v);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        if (c + e < NHW) O[c + e] += __uint_as_float(hi[e]) + __uint_as_float(lo[e]);
+                    for (int e = 0; e < NHW; ++e) O[e] += __uint_as_float(v[e]) + __uint_as_float(v[8 + e]);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < NHW; c += 16) {
+                        uint32_t hi[16], lo[16];
+                        tmem_ld16(obase + c, hi);
+                        tmem_ld16(obase + C::LO + c, lo);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            if (c + e < NHW) O[c + e] += __uint_as_float(hi[e]) + __uint_as_float(lo[e]);
+                    }
                 }
                 tc_fence_before_sync();
                 __syncwarp();
