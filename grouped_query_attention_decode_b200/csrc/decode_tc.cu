@@ -168,8 +168,8 @@ __device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t bytes) {
 // the cache write; nothing else in the kernel reads it.
 //
 // Both kinds of event come in the CTA's walk order, and every wait blocks (a blocking mbarrier
-// wait wakes as soon as its phase completes; an earlier version polled both kinds from one
-// loop with a back-off and took the tickets late).  A piece that ends its unit computes the
+// wait wakes as soon as its phase completes, where polling both kinds from one loop with a
+// back-off takes the tickets late).  A piece that ends its unit computes the
 // unit's last tile -- the patched one -- first, so segment s's patch is due while segment s - 1
 // is still being computed: the ticket of a partial segment is therefore taken after the next
 // segment's patch, which keeps the patch ahead of the scores that wait for it.  No ticket is
