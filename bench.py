@@ -293,6 +293,12 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+def cache_copies(l2_bytes: int, step_bytes: int) -> int:
+    """Copies of the cache that rotate so that a copy is read again only after >= 2 x L2 of
+    other K/V bytes: every step then reads HBM, not L2."""
+    return max(2, min(1024, 1 + math.ceil(2 * l2_bytes / step_bytes)))
+
+
 def percentile(v, p):
     s = sorted(v)
     if not s:
@@ -318,7 +324,7 @@ class Replica:
         self.lengths = x["lengths"].tolist()
         self.ideal = inputs.ideal_kv_bytes(w, self.lengths)
         self.l2_bytes = int(torch.cuda.get_device_properties(dev).L2_cache_size)
-        self.n_copies = n_copies or max(2, min(1024, 1 + math.ceil(2 * self.l2_bytes / self.ideal)))
+        self.n_copies = n_copies or cache_copies(self.l2_bytes, self.ideal)
         self.q = x["q"].to(dev)
         self.kn, self.vn = x["k_new"].to(dev), x["v_new"].to(dev)
         self.block_table = None
